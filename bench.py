@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA lightning-indexer top-k on B200.
+
+One step = one call of the C-ABI entry point over one batch of synthetic
+inputs resident in HBM (the fused indexer/top-k kernel, plus the split merge
+when the plan splits key ranges).  Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own
+independent batch (weak scaling, no data-path collective); the time is the
+max over ranks.  ``--impl reference`` times the CPU oracle on the host cores
+over a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+DEFAULT_CONFIG = "dsa_prefill"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, out_path: str):
+        self.out_path = out_path
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        try:
+            self.f = open(self.out_path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.out_path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(parts)
+                except ValueError:
+                    pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].lower() == "active"})
+        loaded = [x for x in sm if smax and x > 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(wl, inputs_cpu, budget_rows: int):
+    """Time the oracle on an evenly spaced sample of query rows; returns a dict
+    with queries/s extrapolated to the full workload by visible-pair count."""
+    import oracle
+
+    oracle.build()
+    q, w, k, ks = inputs_cpu
+    rows_total = wl.B * wl.S
+    n = min(rows_total, budget_rows)
+    rows = np.unique(np.linspace(0, rows_total - 1, n).round().astype(np.int64))
+    pairs_sample = sum(wl.visible(int(r) % wl.S) for r in rows)
+    pairs_total = wl.visible_pairs()
+    t0 = time.perf_counter()
+    oracle.topk(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m, topk=wl.topk,
+                causal=wl.causal, mode=1 if wl.gated else 0, rows=rows)
+    dt = time.perf_counter() - t0
+    full_time = dt * (pairs_total / max(1, pairs_sample))
+    return {"value": rows_total / full_time, "unit": "queries/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} of {rows_total} query rows evenly spaced in t "
+                      f"({pairs_sample} of {pairs_total} visible pairs); {dt:.2f} s measured, "
+                      f"full-workload time extrapolated by visible-pair count",
+            "seconds": dt}
+
+
+def inputs_for_oracle(wl, inp):
+    return workloads.as_numpy_bits(inp)
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+
+    inp = workloads.make_inputs(wl, device="cpu")
+    cpu = inputs_for_oracle(wl, inp)
+    rows_per_step = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(wl, cpu, max(8, rows_per_step // 8))
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = oracle_sample(wl, cpu, rows_per_step)
+        vals.append(r["value"])
+        secs.append(r["seconds"])
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "indexer queries/s", "value": value, "unit": "queries/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * (wl.B * wl.S) / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl),
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": r["cores"],
+                         "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    del torch
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(wl):
+    return {"workload": wl.name, "B": wl.B, "S": wl.S, "T": wl.T, "H_I": wl.H, "d": wl.d,
+            "m": wl.m, "topk": wl.topk, "causal": wl.causal,
+            "keys": "e4m3+fp32 scale" if wl.key_fp8 else "bf16",
+            "mode": "sigmoid-gate" if wl.gated else "relu-topk",
+            "values": wl.values, "l2": "flushed between timed steps (256 MiB write)",
+            "parallelism": "replicas"}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=256,
+                    help="query rows the oracle computes per reference step")
+    ap.add_argument("--cpu-rows", type=int, default=512,
+                    help="query rows of the CPU-baseline sample (rank 0)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    wl = workloads.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+
+    import lightning_indexer_top_02_b200 as L
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    L.load_library()
+    stream = torch.cuda.current_stream(dev)
+
+    inp = workloads.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
+    q, w, k, ks = inp["q"], inp["w"], inp["k"], inp["k_scale"]
+    out_idx = torch.empty((wl.B, wl.S, wl.topk), dtype=torch.int32, device=dev)
+    out_sc = torch.empty((wl.B, wl.S, wl.topk), dtype=torch.float32, device=dev)
+    mode = 1 if wl.gated else 0
+    a = L.make_args(q, w, k, k_scale=ks, m=wl.m, topk=wl.topk, causal=wl.causal, mode=mode,
+                    out_idx=out_idx, out_score=out_sc)
+    ws_bytes = L.csa_indexer_workspace_size(a)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    import ctypes
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    wsptr = ctypes.c_void_p(ws.data_ptr())
+
+    def step():
+        st = L.csa_indexer_topk_ex(a, wsptr, ws_bytes, sptr)
+        if st != L.CSA_OK:
+            raise L.CsaError(st, "csa_indexer_topk_ex")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if L.csa_last_device_error(sptr) != L.CSA_OK:
+        raise SystemExit("device error during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = None
+    if rank == 0:
+        props = torch.cuda.get_device_properties(dev)
+        gid = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        sampler = ClockSampler(gid, os.path.join(ROOT, "gpurun_out", "bench_clocks.csv"))
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    if L.csa_last_device_error(sptr) != L.CSA_OK:
+        raise SystemExit("device error during the timed region")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    queries = wl.B * wl.S
+    value = queries * world / (ms_per_step / 1000.0)
+    flops = wl.flops()
+    tflops = flops / (ms_per_step / 1000.0) / 1e12
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hw = w.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hks = ks.cpu().pin_memory() if ks is not None else None
+        hidx = torch.empty(out_idx.shape, dtype=torch.int32).pin_memory()
+        hsc = torch.empty(out_sc.shape, dtype=torch.float32).pin_memory()
+        h2d = hq.numel() * hq.element_size() + hw.numel() * 4 + hk.numel() * hk.element_size() + (
+            hks.numel() * 4 if hks is not None else 0)
+        d2h = hidx.numel() * 4 + hsc.numel() * 4
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            w.copy_(hw, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            if hks is not None:
+                ks.copy_(hks, non_blocking=True)
+            step()
+            hidx.copy_(out_idx, non_blocking=True)
+            hsc.copy_(out_sc, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": queries * world / (e_ms / 1000.0), "unit": "queries/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms}
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    timed_s = total_ms / 1000.0
+    sustained = timed_s > 0.5
+    peak = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
+    nsplit_launches = 1
+    roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                "frac": tflops / peak if peak else None, "traffic": None,
+                "peak_source": f"{peak_src} bf16 dense ({'sustained' if sustained else 'burst'})",
+                "kernel": "indexer_topk_kernel (+ split merge when the plan splits)",
+                "algorithmic_flops_per_launch": flops}
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu_inputs = inputs_for_oracle(wl, {"q": q, "w": w, "k": k, "k_scale": ks})
+        r = oracle_sample(wl, cpu_inputs, args.cpu_rows)
+        cpu = {k_: r[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
+
+    line = {
+        "metric": "indexer queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_dict(wl), "tflops": tflops,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": args.steps * nsplit_launches,
+        "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
+                    "max": max(step_ms)},
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

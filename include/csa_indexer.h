@@ -1,0 +1,137 @@
+/*
+ * csa_indexer.h -- C ABI of the B200 (sm_100a) CSA lightning-indexer top-k.
+ *
+ * The operation ("StreamIndex: Memory-Bounded Compressed Sparse Attention via
+ * Streaming Top-k", abstract: a lightning indexer scores compressed keys, the
+ * top-k are selected per query, and the full [B,S,H_I,T] score tensor is
+ * never materialised):
+ *
+ *   for every batch b and query row i, with absolute position t = i + q_offset,
+ *     key s (covering tokens [s*m, (s+1)*m)) is visible iff !causal or
+ *     (s+1)*m - 1 <= t, and
+ *       I[t,s] = sum_h w[b,i,h] * ReLU( sum_j q[b,i,h,j] * k[b,s,j] )
+ *     (FP8 keys: k[b,s,j] = k_scale[b,s] * E4M3(k8[b,s,j]))
+ *   CSA_MODE_TOPK: return the min(topk, #visible) visible keys with the
+ *     largest I, ordered by I descending, equal scores by ascending s.
+ *   CSA_MODE_GATE: keep only visible keys with sigmoid(I) > 0.5, i.e. I > 0
+ *     ("FlashMemory-DeepSeek-V4: Lightning Index Ultra-Long Context via
+ *     Lookahead Sparse Attention", "What carries the argument": a sigmoid
+ *     gate with a fixed 0.5 threshold in place of a fixed top-k), at most
+ *     topk of them, chosen and ordered as in CSA_MODE_TOPK.
+ *   Unused output slots hold index -1 and score -inf.  A zero score is +0.0.
+ *
+ * Layouts (all contiguous, row-major, DEVICE memory owned by the caller):
+ *   q         [B, S, H_I, d]  bfloat16
+ *   w         [B, S, H_I]     float32
+ *   k         [B, T, d]       bfloat16 (CSA_KEY_BF16) or E4M3 bytes (CSA_KEY_E4M3)
+ *   k_scale   [B, T]          float32, > 0 (CSA_KEY_E4M3 only)
+ *   out_idx   [B, S, topk]    int32, key indices in [0, T) or -1
+ *   out_score [B, S, topk]    float32
+ * q, k, k_scale and the outputs must be 16-byte aligned.  Inputs must be
+ * finite; NaN or Inf inputs give unspecified (but memory-safe) results.
+ *
+ * Supported shapes: H_I a power of two in [1, 256]; d in {32, 64, 128};
+ * 1 <= topk <= 2048; m >= 1; T, S < 2^31.  Anything else returns
+ * CSA_ERR_UNSUPPORTED before any launch.  There is no CPU fallback.
+ *
+ * All calls are stream-ordered on `stream`: they enqueue work and return
+ * without synchronising.  Errors are returned as status codes; no call throws
+ * across this boundary.  Arguments are validated before any launch
+ * (CSA_ERR_INVALID_ARG / CSA_ERR_UNSUPPORTED leave the outputs untouched).
+ * Every device-side wait is bounded; a wait that runs out records a timeout
+ * that csa_last_device_error() reports, and the kernel exits cleanly.
+ */
+#ifndef CSA_INDEXER_H
+#define CSA_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, misaligned pointer */
+    CSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes listed above       */
+    CSA_ERR_WORKSPACE = 3,   /* caller workspace smaller than csa_indexer_workspace_size  */
+    CSA_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, allocation, ...)      */
+    CSA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see csa_last_device_error) */
+} csa_status_t;
+
+typedef enum { CSA_KEY_BF16 = 0, CSA_KEY_E4M3 = 1 } csa_key_dtype_t;
+typedef enum { CSA_MODE_TOPK = 0, CSA_MODE_GATE = 1 } csa_mode_t;
+
+/* Full argument set of one indexer call.  Pointers are device pointers. */
+typedef struct {
+    const void *q;         /* [B,S,H_I,d] bf16                                 */
+    const float *w;        /* [B,S,H_I] fp32                                   */
+    const void *k;         /* [B,T,d] bf16 or E4M3 bytes                       */
+    const float *k_scale;  /* [B,T] fp32 > 0 for CSA_KEY_E4M3, else NULL       */
+    int B, S, T, H_I, d, m, topk;
+    int causal;            /* 0: every key visible; 1: the causal rule above   */
+    int key_dtype;         /* csa_key_dtype_t                                  */
+    int mode;              /* csa_mode_t                                       */
+    long long q_offset;    /* absolute position of query row 0; < 0 selects the
+                              default max(0, T*m - S) (queries end where the
+                              keys' token span ends)                           */
+    int num_splits;        /* key-range splits per query block; 0 = automatic  */
+    int32_t *out_idx;      /* [B,S,topk]                                       */
+    float *out_score;      /* [B,S,topk]                                       */
+} csa_args_t;
+
+/*
+ * The spec entry point: bf16 q and k, ReLU top-k, default q_offset.
+ * Needs scratch memory, which it takes with cudaMallocAsync on `stream` and
+ * returns with cudaFreeAsync on the same stream (stream-ordered; no sync).
+ */
+csa_status_t csa_indexer_topk(const void *q, const float *w, const void *k,
+                              int B, int S, int T, int H_I, int d, int m, int topk,
+                              int causal, int32_t *out_idx, float *out_score,
+                              cudaStream_t stream);
+
+/*
+ * Bytes of device scratch csa_indexer_topk_ex needs for these arguments
+ * (depends on shapes, topk and the device's SM count, not on the data).
+ * Returns 0 for arguments that csa_indexer_topk_ex would reject.
+ */
+size_t csa_indexer_workspace_size(const csa_args_t *args);
+
+/*
+ * Extended entry point: any key dtype and mode, explicit q_offset and split
+ * count.  `workspace` is caller-owned device memory of at least
+ * csa_indexer_workspace_size(args) bytes, 256-byte aligned, used only for
+ * the duration of the enqueued work; pass NULL to have the call allocate and
+ * free it stream-ordered on `stream` (cudaMallocAsync/cudaFreeAsync).
+ * Two calls that share a workspace must not overlap on the GPU.
+ */
+csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
+
+/* Static text for a status code. */
+const char *csa_status_string(csa_status_t status);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the device error word that
+ * bounded waits set when they run out on the current device:
+ * CSA_OK, CSA_ERR_TIMEOUT, or CSA_ERR_CUDA if the synchronisation failed.
+ */
+csa_status_t csa_last_device_error(cudaStream_t stream);
+
+/*
+ * Cycle budget of every bounded device-side wait for later launches on the
+ * calling thread's current device (default 4e9 cycles, about two seconds).
+ * Tests shrink it to make a wait run out on purpose.  0 restores the default.
+ */
+void csa_set_wait_limit(unsigned long long cycles);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int csa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_INDEXER_H */

@@ -1,0 +1,450 @@
+// csa_indexer.cu -- host side of the C ABI declared in include/csa_indexer.h:
+// argument validation, work planning (query blocks, sub-blocks, key splits,
+// pipeline depth, candidate capacity), TMA descriptors, workspace layout and
+// launches of the fused indexer/top-k kernel and the split merge.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "csa_indexer.h"
+#include "indexer_kernel.cuh"
+
+namespace {
+
+using csa::Params;
+
+constexpr int kVersion = 100; // 0.1.0
+constexpr int kSmemLimit = 232448; // 227 KB of dynamic shared memory per CTA on sm_100
+constexpr unsigned long long kDefaultWaitLimit = 4000000000ull;
+
+unsigned long long g_wait_limit = kDefaultWaitLimit;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int pow2_ceil(long long x)
+{
+    int p = 1;
+    while (p < x && p < (1 << 30))
+        p <<= 1;
+    return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Plan {
+    Params p;
+    int grid;
+    size_t ws_cand, ws_part, ws_total;
+};
+
+csa_status_t validate(const csa_args_t *a)
+{
+    if (!a)
+        return CSA_ERR_INVALID_ARG;
+    if (a->B < 0 || a->S < 0 || a->T < 0 || a->H_I <= 0 || a->d <= 0 || a->m <= 0 ||
+        a->topk <= 0)
+        return CSA_ERR_INVALID_ARG;
+    if ((a->causal != 0 && a->causal != 1) || (a->mode != CSA_MODE_TOPK && a->mode != CSA_MODE_GATE) ||
+        (a->key_dtype != CSA_KEY_BF16 && a->key_dtype != CSA_KEY_E4M3))
+        return CSA_ERR_INVALID_ARG;
+    if (static_cast<long long>(a->B) * a->S == 0)
+        return CSA_OK;
+    if (!a->q || !a->w || !a->out_idx || !a->out_score)
+        return CSA_ERR_INVALID_ARG;
+    if (a->T > 0 && !a->k)
+        return CSA_ERR_INVALID_ARG;
+    if (a->key_dtype == CSA_KEY_E4M3 && a->T > 0 && !a->k_scale)
+        return CSA_ERR_INVALID_ARG;
+    if (!aligned(a->q, 16) || (a->k && !aligned(a->k, 16)) || !aligned(a->w, 4) ||
+        !aligned(a->out_idx, 4) || !aligned(a->out_score, 4) ||
+        (a->k_scale && !aligned(a->k_scale, 4)))
+        return CSA_ERR_INVALID_ARG;
+    if (!is_pow2(a->H_I) || a->H_I > 256)
+        return CSA_ERR_UNSUPPORTED;
+    if (a->d != 32 && a->d != 64 && a->d != 128)
+        return CSA_ERR_UNSUPPORTED;
+    if (a->topk > csa::kMaxTopk)
+        return CSA_ERR_UNSUPPORTED;
+    if (a->key_dtype == CSA_KEY_E4M3)
+        return CSA_ERR_UNSUPPORTED; // FP8 keys: not yet built
+    const long long rows_q = static_cast<long long>(a->B) * a->S * a->H_I;
+    const long long rows_k = static_cast<long long>(a->B) * a->T;
+    if (rows_q >= (1ll << 31) || rows_k >= (1ll << 31))
+        return CSA_ERR_UNSUPPORTED;
+    return CSA_OK;
+}
+
+int device_sms()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
+}
+
+// Number of key tiles the heaviest query block of a batch touches.
+int max_tiles(const csa_args_t *a, long long q_offset)
+{
+    long long nvis = a->T;
+    if (a->causal) {
+        const long long t = static_cast<long long>(a->S) - 1 + q_offset;
+        nvis = (t + 1) / a->m;
+        if (nvis > a->T)
+            nvis = a->T;
+        if (nvis < 0)
+            nvis = 0;
+    }
+    return static_cast<int>((nvis + csa::kTileKeys - 1) / csa::kTileKeys);
+}
+
+csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
+{
+    Params p;
+    std::memset(&p, 0, sizeof p);
+    p.B = a->B;
+    p.S = a->S;
+    p.T = a->T;
+    p.H = a->H_I;
+    p.d = a->d;
+    p.m = a->m;
+    p.topk = a->topk;
+    p.causal = a->causal;
+    p.mode = a->mode;
+    p.key_fp8 = a->key_dtype == CSA_KEY_E4M3;
+    p.q_offset = a->q_offset >= 0 ? a->q_offset
+                                  : (static_cast<long long>(a->T) * a->m > a->S
+                                         ? static_cast<long long>(a->T) * a->m - a->S
+                                         : 0);
+    p.row_bytes = a->d * 2 < 128 ? a->d * 2 : 128;
+    p.n_chunks = a->d * 2 / p.row_bytes;
+
+    // Query sub-block: as many queries as fill 256 MMA columns, no more than S
+    // needs, and at least 32 columns (one TMEM load of the epilogue).
+    int qps = 256 / p.H;
+    if (qps > pow2_ceil(p.S))
+        qps = pow2_ceil(p.S);
+    if (qps * p.H < 32)
+        qps = 32 / p.H;
+    p.qps = qps;
+    p.N = qps * p.H;
+
+    p.cap = 2 * p.topk;
+    if (p.cap < p.topk + 256)
+        p.cap = p.topk + 256;
+    p.cap = (p.cap + 127) / 128 * 128;
+    if (p.cap > csa::kEpiThreads * csa::kEpt)
+        return CSA_ERR_UNSUPPORTED;
+    p.slack = (p.cap - csa::kTileKeys - p.topk) / 2;
+
+    const int k_stage = csa::kTileKeys * p.d * 2;
+    for (int nsub = (p.S > qps ? 2 : 1); nsub >= 1; --nsub) {
+        p.nsub = nsub;
+        p.qpb = nsub * qps;
+        int off = 0;
+        p.off_q = off;
+        off += nsub * p.N * p.d * 2;
+        p.off_k = off;
+        const int fixed_after_k = 0;
+        (void)fixed_after_k;
+        // everything after the key stages
+        int tail = 0;
+        const int sort_bytes = csa::pow2_at_least(p.topk) * 8;
+        tail += sort_bytes;
+        tail += p.qpb * p.H * 4;
+        tail = (tail + 15) / 16 * 16;
+        tail += p.qpb * static_cast<int>(sizeof(csa::QueryState));
+        tail += static_cast<int>(sizeof(csa::GroupScratch));
+        tail = (tail + 15) / 16 * 16;
+        tail += static_cast<int>(sizeof(csa::Barriers));
+        const int budget = kSmemLimit - 1024 - off - tail;
+        int stages = budget / k_stage;
+        if (stages > csa::kMaxStages)
+            stages = csa::kMaxStages;
+        if (stages < 2)
+            continue;
+        p.stages = stages;
+        off += stages * k_stage;
+        p.off_sort = off;
+        off += sort_bytes;
+        p.off_w = off;
+        off += p.qpb * p.H * 4;
+        off = (off + 15) / 16 * 16;
+        p.off_state = off;
+        off += p.qpb * static_cast<int>(sizeof(csa::QueryState));
+        p.off_scratch = off;
+        off += static_cast<int>(sizeof(csa::GroupScratch));
+        off = (off + 15) / 16 * 16;
+        p.off_bar = off;
+        off += static_cast<int>(sizeof(csa::Barriers));
+        p.smem_bytes = off + 1024;
+        // More than half of the SM's shared memory: one CTA per SM, so the
+        // CTA's 512-column TMEM allocation never waits on a neighbour.
+        if (p.smem_bytes < kSmemLimit / 2 + 1024)
+            p.smem_bytes = kSmemLimit / 2 + 1024;
+        break;
+    }
+    if (p.stages < 2)
+        return CSA_ERR_UNSUPPORTED;
+    p.nqb = (p.S + p.qpb - 1) / p.qpb;
+
+    // Key-range splits: only when there are too few query blocks to fill the
+    // GPU; pick the count with the best last-wave occupancy.
+    const long long items_base = static_cast<long long>(p.B) * p.nqb;
+    int nsplit = 1;
+    if (a->num_splits > 0) {
+        nsplit = a->num_splits;
+    } else if (items_base < 4ll * sms) {
+        const int tiles = max_tiles(a, p.q_offset);
+        int max_split = 8192 / p.topk;
+        if (max_split > 16)
+            max_split = 16;
+        if (max_split > tiles)
+            max_split = tiles;
+        double best = -1.0;
+        for (int s = 1; s <= max_split; ++s) {
+            const long long items = items_base * s;
+            const long long waves = (items + sms - 1) / sms;
+            const double eff = static_cast<double>(items) / static_cast<double>(waves * sms);
+            const double score = eff - 0.01 * (s - 1);
+            if (score > best + 1e-9) {
+                best = score;
+                nsplit = s;
+            }
+        }
+    }
+    if (nsplit < 1 || static_cast<long long>(nsplit) * p.topk > 8192)
+        return CSA_ERR_UNSUPPORTED;
+    p.nsplit = nsplit;
+    const long long items = items_base * nsplit;
+    if (items >= (1ll << 31))
+        return CSA_ERR_UNSUPPORTED;
+    p.n_items = static_cast<int>(items);
+
+    Plan plan;
+    plan.grid = p.n_items < sms ? p.n_items : sms;
+    if (plan.grid < 1)
+        plan.grid = 1;
+    plan.ws_cand = align256(static_cast<size_t>(plan.grid) * p.qpb * p.cap * 8);
+    plan.ws_part = nsplit > 1
+                       ? align256(static_cast<size_t>(p.B) * p.S * nsplit * p.topk * 8)
+                       : 0;
+    plan.ws_total = plan.ws_cand + plan.ws_part;
+    plan.p = p;
+    *out = plan;
+    return CSA_OK;
+}
+
+bool make_tmap(CUtensorMap *tm, CUtensorMapDataType dt, const void *base, long long rows, int cols,
+               int box_cols, int box_rows, CUtensorMapSwizzle swz)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estride[2] = {1, 1};
+    return enc(tm, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+__global__ void pad_outputs_kernel(int32_t *idx, float *score, long long n)
+{
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        idx[i] = -1;
+        score[i] = -__int_as_float(0x7f800000);
+    }
+}
+
+csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_t stream)
+{
+    Params p = plan.p;
+    p.w = a->w;
+    p.k_scale = a->k_scale;
+    p.out_idx = a->out_idx;
+    p.out_score = a->out_score;
+    p.cand = reinterpret_cast<uint64_t *>(ws);
+    p.part = plan.ws_part ? reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(ws) + plan.ws_cand)
+                          : nullptr;
+    p.wait_limit = static_cast<long long>(g_wait_limit);
+
+    CUtensorMap tmQ, tmK;
+    const CUtensorMapSwizzle swz =
+        p.row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapDataType qdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap(&tmQ, qdt, a->q, static_cast<long long>(p.B) * p.S * p.H, p.d, p.row_bytes / 2,
+                   p.N, swz))
+        return CSA_ERR_CUDA;
+    if (!make_tmap(&tmK, qdt, a->k, static_cast<long long>(p.B) * p.T, p.d, p.row_bytes / 2,
+                   csa::kTileKeys, swz))
+        return CSA_ERR_CUDA;
+
+    const bool ge32 = p.H >= 32;
+    auto kern = ge32 ? csa::indexer_topk_kernel<true> : csa::indexer_topk_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes) !=
+        cudaSuccess)
+        return CSA_ERR_CUDA;
+    kern<<<plan.grid, csa::kThreads, p.smem_bytes, stream>>>(tmQ, tmK, p);
+    if (cudaGetLastError() != cudaSuccess)
+        return CSA_ERR_CUDA;
+    if (p.nsplit > 1) {
+        const int rows = p.B * p.S;
+        const int sms = device_sms();
+        int grid = rows < sms * 8 ? rows : sms * 8;
+        csa::merge_splits_kernel<<<grid, csa::kMergeThreads, 0, stream>>>(
+            p.part, rows, p.nsplit, p.topk, p.out_idx, p.out_score);
+        if (cudaGetLastError() != cudaSuccess)
+            return CSA_ERR_CUDA;
+    }
+    return CSA_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+size_t csa_indexer_workspace_size(const csa_args_t *args)
+{
+    if (validate(args) != CSA_OK)
+        return 0;
+    if (static_cast<long long>(args->B) * args->S == 0 || args->T == 0)
+        return 0;
+    const int sms = device_sms();
+    if (sms <= 0)
+        return 0;
+    Plan plan;
+    if (make_plan(args, sms, &plan) != CSA_OK)
+        return 0;
+    return plan.ws_total;
+}
+
+csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream)
+{
+    csa_status_t st = validate(args);
+    if (st != CSA_OK)
+        return st;
+    const long long rows = static_cast<long long>(args->B) * args->S;
+    if (rows == 0)
+        return CSA_OK;
+    if (args->T == 0) {
+        pad_outputs_kernel<<<256, 256, 0, stream>>>(args->out_idx, args->out_score,
+                                                    rows * args->topk);
+        return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+    }
+    const int sms = device_sms();
+    if (sms <= 0)
+        return CSA_ERR_CUDA;
+    Plan plan;
+    st = make_plan(args, sms, &plan);
+    if (st != CSA_OK)
+        return st;
+    if (workspace) {
+        if (workspace_bytes < plan.ws_total)
+            return CSA_ERR_WORKSPACE;
+        if (!aligned(workspace, 256))
+            return CSA_ERR_INVALID_ARG;
+        return launch(args, plan, workspace, stream);
+    }
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, plan.ws_total, stream) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    st = launch(args, plan, ws, stream);
+    if (cudaFreeAsync(ws, stream) != cudaSuccess && st == CSA_OK)
+        st = CSA_ERR_CUDA;
+    return st;
+}
+
+csa_status_t csa_indexer_topk(const void *q, const float *w, const void *k, int B, int S, int T,
+                              int H_I, int d, int m, int topk, int causal, int32_t *out_idx,
+                              float *out_score, cudaStream_t stream)
+{
+    csa_args_t a;
+    std::memset(&a, 0, sizeof a);
+    a.q = q;
+    a.w = w;
+    a.k = k;
+    a.k_scale = nullptr;
+    a.B = B;
+    a.S = S;
+    a.T = T;
+    a.H_I = H_I;
+    a.d = d;
+    a.m = m;
+    a.topk = topk;
+    a.causal = causal;
+    a.key_dtype = CSA_KEY_BF16;
+    a.mode = CSA_MODE_TOPK;
+    a.q_offset = -1;
+    a.num_splits = 0;
+    a.out_idx = out_idx;
+    a.out_score = out_score;
+    return csa_indexer_topk_ex(&a, nullptr, 0, stream);
+}
+
+const char *csa_status_string(csa_status_t status)
+{
+    switch (status) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case CSA_ERR_WORKSPACE: return "workspace too small";
+    case CSA_ERR_CUDA: return "CUDA runtime error";
+    case CSA_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+csa_status_t csa_last_device_error(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    int h[4] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(h, csa::g_csa_error, sizeof h) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    if (h[0] == 0)
+        return CSA_OK;
+    const int zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(csa::g_csa_error, zero, sizeof zero) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    return h[0] == csa::kErrTimeout ? CSA_ERR_TIMEOUT : CSA_ERR_CUDA;
+}
+
+void csa_set_wait_limit(unsigned long long cycles)
+{
+    g_wait_limit = cycles ? cycles : kDefaultWaitLimit;
+}
+
+int csa_version(void) { return kVersion; }
+
+} // extern "C"
