@@ -226,7 +226,8 @@ def main():
     mode = 1 if wl.gated else 0
     a = L.make_args(q, w, k, k_scale=ks, m=wl.m, topk=wl.topk, causal=wl.causal, mode=mode,
                     out_idx=out_idx, out_score=out_sc)
-    ws_bytes = L.csa_indexer_workspace_size(a)
+    plan = L.csa_indexer_plan(a)
+    ws_bytes = plan.workspace_bytes
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     import ctypes
@@ -335,7 +336,6 @@ def main():
     timed_s = total_ms / 1000.0
     sustained = timed_s > 0.5
     peak = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
-    nsplit_launches = 1
     roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                 "frac": tflops / peak if peak else None, "traffic": None,
                 "peak_source": f"{peak_src} bf16 dense ({'sustained' if sustained else 'burst'})",
@@ -353,7 +353,8 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": config_dict(wl), "tflops": tflops,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
-        "gpu_launches": args.steps * nsplit_launches,
+        "gpu_launches": args.steps * plan.launches,
+        "plan": plan.as_dict(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
                     "max": max(step_ms)},
     }

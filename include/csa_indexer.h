@@ -110,6 +110,27 @@ size_t csa_indexer_workspace_size(const csa_args_t *args);
 csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
                                  size_t workspace_bytes, cudaStream_t stream);
 
+/* How csa_indexer_topk_ex would run a call (for benchmarks and tests). */
+typedef struct {
+    int grid;              /* CTAs of the fused kernel (persistent, <= SM count) */
+    int threads;           /* threads per CTA                                    */
+    int smem_bytes;        /* dynamic shared memory per CTA                      */
+    int stages;            /* key-tile pipeline depth                            */
+    int queries_per_block; /* queries one work item covers                       */
+    int num_splits;        /* key-range splits per query block                   */
+    int launches;          /* kernel launches per call (1, or 2 with a merge)    */
+    size_t workspace_bytes;
+} csa_plan_t;
+
+/*
+ * Fills *plan for these arguments on the current device without launching
+ * anything.  Returns the status csa_indexer_topk_ex would return before
+ * launching (CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA
+ * when no device is present).  For B*S == 0 or T == 0 the plan is all zeros
+ * apart from `launches` (0 or 1).
+ */
+csa_status_t csa_indexer_plan(const csa_args_t *args, csa_plan_t *plan);
+
 /* Static text for a status code. */
 const char *csa_status_string(csa_status_t status);
 
@@ -121,8 +142,8 @@ const char *csa_status_string(csa_status_t status);
 csa_status_t csa_last_device_error(cudaStream_t stream);
 
 /*
- * Cycle budget of every bounded device-side wait for later launches on the
- * calling thread's current device (default 4e9 cycles, about two seconds).
+ * Cycle budget of every bounded device-side wait for later launches from this
+ * process (default 4e9 cycles, about two seconds at the B200's clocks).
  * Tests shrink it to make a wait run out on purpose.  0 restores the default.
  */
 void csa_set_wait_limit(unsigned long long cycles);

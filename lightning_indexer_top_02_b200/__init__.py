@@ -31,7 +31,8 @@ CSA_MODE_TOPK = 0
 CSA_MODE_GATE = 1
 
 EXPORTS = ("csa_indexer_topk", "csa_indexer_topk_ex", "csa_indexer_workspace_size",
-           "csa_status_string", "csa_last_device_error", "csa_set_wait_limit", "csa_version")
+           "csa_indexer_plan", "csa_status_string", "csa_last_device_error",
+           "csa_set_wait_limit", "csa_version")
 
 
 class CsaError(RuntimeError):
@@ -50,6 +51,16 @@ class CsaArgs(ctypes.Structure):
         ("q_offset", ctypes.c_longlong), ("num_splits", ctypes.c_int),
         ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
     ]
+
+
+class CsaPlan(ctypes.Structure):
+    _fields_ = [("grid", ctypes.c_int), ("threads", ctypes.c_int), ("smem_bytes", ctypes.c_int),
+                ("stages", ctypes.c_int), ("queries_per_block", ctypes.c_int),
+                ("num_splits", ctypes.c_int), ("launches", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
 
 
 _lib = None
@@ -71,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.csa_indexer_topk_ex.restype = I
     lib.csa_indexer_workspace_size.argtypes = [ctypes.POINTER(CsaArgs)]
     lib.csa_indexer_workspace_size.restype = ctypes.c_size_t
+    lib.csa_indexer_plan.argtypes = [ctypes.POINTER(CsaArgs), ctypes.POINTER(CsaPlan)]
+    lib.csa_indexer_plan.restype = I
     lib.csa_status_string.argtypes = [I]
     lib.csa_status_string.restype = ctypes.c_char_p
     lib.csa_last_device_error.argtypes = [P]
@@ -98,6 +111,14 @@ def csa_indexer_topk_ex(args: CsaArgs, workspace_ptr, workspace_bytes: int, stre
 
 def csa_indexer_workspace_size(args: CsaArgs) -> int:
     return load_library().csa_indexer_workspace_size(ctypes.byref(args))
+
+
+def csa_indexer_plan(args: CsaArgs) -> CsaPlan:
+    plan = CsaPlan()
+    st = load_library().csa_indexer_plan(ctypes.byref(args), ctypes.byref(plan))
+    if st != CSA_OK:
+        raise CsaError(st, "csa_indexer_plan")
+    return plan
 
 
 def csa_status_string(status: int) -> str:

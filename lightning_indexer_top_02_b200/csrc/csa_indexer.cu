@@ -348,6 +348,38 @@ size_t csa_indexer_workspace_size(const csa_args_t *args)
     return plan.ws_total;
 }
 
+csa_status_t csa_indexer_plan(const csa_args_t *args, csa_plan_t *out)
+{
+    if (!out)
+        return CSA_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof *out);
+    csa_status_t st = validate(args);
+    if (st != CSA_OK)
+        return st;
+    if (static_cast<long long>(args->B) * args->S == 0)
+        return CSA_OK;
+    if (args->T == 0) {
+        out->launches = 1;
+        return CSA_OK;
+    }
+    const int sms = device_sms();
+    if (sms <= 0)
+        return CSA_ERR_CUDA;
+    Plan plan;
+    st = make_plan(args, sms, &plan);
+    if (st != CSA_OK)
+        return st;
+    out->grid = plan.grid;
+    out->threads = csa::kThreads;
+    out->smem_bytes = plan.p.smem_bytes;
+    out->stages = plan.p.stages;
+    out->queries_per_block = plan.p.qpb;
+    out->num_splits = plan.p.nsplit;
+    out->launches = plan.p.nsplit > 1 ? 2 : 1;
+    out->workspace_bytes = plan.ws_total;
+    return CSA_OK;
+}
+
 csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace, size_t workspace_bytes,
                                  cudaStream_t stream)
 {
@@ -448,3 +480,4 @@ void csa_set_wait_limit(unsigned long long cycles)
 int csa_version(void) { return kVersion; }
 
 } // extern "C"
+
