@@ -110,6 +110,29 @@ size_t csa_indexer_workspace_size(const csa_args_t *args);
 csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
                                  size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Same operation as csa_indexer_topk_ex, for callers that cannot allocate
+ * device memory while they run: latency-critical serving loops that must not
+ * risk cudaMalloc's device-wide synchronisation mid-step, and hosts whose
+ * memory budget is fixed up front and that forbid allocations outside their
+ * own pool.  The paper has no counterpart; this is a deployment variant.
+ *
+ * The call allocates nothing.  Its scratch is one fixed 64 MiB device array
+ * inside this library (CSA_NOALLOC_SCRATCH_BYTES), which every GPU that loads
+ * the library holds until the process exits.  The caller still passes all
+ * inputs and outputs.  The first call on each device looks up that array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  If a full grid's scratch does not fit, the call runs fewer
+ * persistent CTAs; if the shape needs more than the array even then (large
+ * B*S*topk with key-range splits), it returns CSA_ERR_WORKSPACE and launches
+ * nothing.  All calls share the one array and nothing in it needs to start at
+ * zero, but two calls that overlap on the GPU (different streams, or
+ * different host threads) race on it and give undefined results: serialise
+ * them.
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES (64ull << 20)
+csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStream_t stream);
+
 /* How csa_indexer_topk_ex would run a call (for benchmarks and tests). */
 typedef struct {
     int grid;              /* CTAs of the fused kernel (persistent, <= SM count) */

@@ -31,8 +31,8 @@ CSA_MODE_TOPK = 0
 CSA_MODE_GATE = 1
 
 EXPORTS = ("csa_indexer_topk", "csa_indexer_topk_ex", "csa_indexer_workspace_size",
-           "csa_indexer_plan", "csa_status_string", "csa_last_device_error",
-           "csa_set_wait_limit", "csa_version")
+           "csa_indexer_plan", "csa_indexer_topk_noalloc", "csa_status_string",
+           "csa_last_device_error", "csa_set_wait_limit", "csa_version")
 
 
 class CsaError(RuntimeError):
@@ -82,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.csa_indexer_topk_ex.restype = I
     lib.csa_indexer_workspace_size.argtypes = [ctypes.POINTER(CsaArgs)]
     lib.csa_indexer_workspace_size.restype = ctypes.c_size_t
+    lib.csa_indexer_topk_noalloc.argtypes = [ctypes.POINTER(CsaArgs), P]
+    lib.csa_indexer_topk_noalloc.restype = I
     lib.csa_indexer_plan.argtypes = [ctypes.POINTER(CsaArgs), ctypes.POINTER(CsaPlan)]
     lib.csa_indexer_plan.restype = I
     lib.csa_status_string.argtypes = [I]
@@ -111,6 +113,11 @@ def csa_indexer_topk_ex(args: CsaArgs, workspace_ptr, workspace_bytes: int, stre
 
 def csa_indexer_workspace_size(args: CsaArgs) -> int:
     return load_library().csa_indexer_workspace_size(ctypes.byref(args))
+
+
+def csa_indexer_topk_noalloc(args: CsaArgs, stream_ptr) -> int:
+    """The allocation-free entry point (fixed in-library scratch; see the header)."""
+    return load_library().csa_indexer_topk_noalloc(ctypes.byref(args), stream_ptr)
 
 
 def csa_indexer_plan(args: CsaArgs) -> CsaPlan:

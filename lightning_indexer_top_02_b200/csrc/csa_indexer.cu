@@ -481,3 +481,83 @@ int csa_version(void) { return kVersion; }
 
 } // extern "C"
 
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.
+//
+// Some callers cannot allocate device memory at call time: serving loops that
+// must not risk cudaMalloc's device-wide synchronisation in the middle of a
+// latency-critical step, and hosts whose memory budget is fixed up front and
+// that forbid allocations outside their own pool.  For them the scratch this
+// operation needs lives in one fixed array below, created with the library's
+// module on every GPU that loads it and held until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20; // 64 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the array's name as a device pointer).
+csa_status_t noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return CSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return CSA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return CSA_OK;
+}
+
+} // namespace
+
+extern "C" csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStream_t stream)
+{
+    csa_status_t st = validate(args);
+    if (st != CSA_OK)
+        return st;
+    const long long rows = static_cast<long long>(args->B) * args->S;
+    if (rows == 0)
+        return CSA_OK;
+    if (args->T == 0) {
+        pad_outputs_kernel<<<256, 256, 0, stream>>>(args->out_idx, args->out_score,
+                                                    rows * args->topk);
+        return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+    }
+    const int sms = device_sms();
+    if (sms <= 0)
+        return CSA_ERR_CUDA;
+    Plan plan;
+    st = make_plan(args, sms, &plan);
+    if (st != CSA_OK)
+        return st;
+    // The per-CTA candidate lists scale with the grid: run fewer persistent
+    // CTAs when a full grid's lists do not fit next to the split partials.
+    if (plan.ws_total > kNoAllocScratchBytes) {
+        const size_t per_cta = static_cast<size_t>(plan.p.qpb) * plan.p.cap * 8;
+        if (plan.ws_part + 256 > kNoAllocScratchBytes)
+            return CSA_ERR_WORKSPACE;
+        const size_t fit = (kNoAllocScratchBytes - plan.ws_part - 256) / per_cta;
+        if (fit < 1)
+            return CSA_ERR_WORKSPACE;
+        plan.grid = static_cast<int>(fit < static_cast<size_t>(plan.grid) ? fit : plan.grid);
+        plan.ws_cand = align256(static_cast<size_t>(plan.grid) * per_cta);
+        plan.ws_total = plan.ws_cand + plan.ws_part;
+        if (plan.ws_total > kNoAllocScratchBytes)
+            return CSA_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != CSA_OK)
+        return st;
+    return launch(args, plan, scratch, stream);
+}
