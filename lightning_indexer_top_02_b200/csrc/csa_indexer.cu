@@ -146,7 +146,7 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
     p.row_bytes = a->d * 2 < 128 ? a->d * 2 : 128;
     p.n_chunks = a->d * 2 / p.row_bytes;
 
-    // Query sub-block: as many queries as fill 256 MMA columns, no more than S
+    // Query block: as many queries as fill 256 MMA columns, no more than S
     // needs, and at least 32 columns (one TMEM load of the epilogue).
     int qps = 256 / p.H;
     if (qps > pow2_ceil(p.S))
@@ -155,65 +155,56 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
         qps = 32 / p.H;
     p.qps = qps;
     p.N = qps * p.H;
+    // Two epilogue warpgroups split the queries when each half still spans
+    // whole 32-column TMEM loads.
+    p.n_wg = (qps >= 2 && p.N >= 64) ? 2 : 1;
+    p.qpw = qps / p.n_wg;
 
     p.cap = 2 * p.topk;
     if (p.cap < p.topk + 256)
         p.cap = p.topk + 256;
     p.cap = (p.cap + 127) / 128 * 128;
-    if (p.cap > csa::kEpiThreads * csa::kEpt)
+    if (p.cap > csa::kGroupThreads * csa::kEpt)
         return CSA_ERR_UNSUPPORTED;
     p.slack = (p.cap - csa::kTileKeys - p.topk) / 2;
 
     const int k_stage = csa::kTileKeys * p.d * 2;
-    for (int nsub = (p.S > qps ? 2 : 1); nsub >= 1; --nsub) {
-        p.nsub = nsub;
-        p.qpb = nsub * qps;
-        int off = 0;
-        p.off_q = off;
-        off += nsub * p.N * p.d * 2;
-        p.off_k = off;
-        const int fixed_after_k = 0;
-        (void)fixed_after_k;
-        // everything after the key stages
-        int tail = 0;
-        const int sort_bytes = csa::pow2_at_least(p.topk) * 8;
-        tail += sort_bytes;
-        tail += p.qpb * p.H * 4;
-        tail = (tail + 15) / 16 * 16;
-        tail += p.qpb * static_cast<int>(sizeof(csa::QueryState));
-        tail += static_cast<int>(sizeof(csa::GroupScratch));
-        tail = (tail + 15) / 16 * 16;
-        tail += static_cast<int>(sizeof(csa::Barriers));
-        const int budget = kSmemLimit - 1024 - off - tail;
-        int stages = budget / k_stage;
-        if (stages > csa::kMaxStages)
-            stages = csa::kMaxStages;
-        if (stages < 2)
-            continue;
-        p.stages = stages;
-        off += stages * k_stage;
-        p.off_sort = off;
-        off += sort_bytes;
-        p.off_w = off;
-        off += p.qpb * p.H * 4;
-        off = (off + 15) / 16 * 16;
-        p.off_state = off;
-        off += p.qpb * static_cast<int>(sizeof(csa::QueryState));
-        p.off_scratch = off;
-        off += static_cast<int>(sizeof(csa::GroupScratch));
-        off = (off + 15) / 16 * 16;
-        p.off_bar = off;
-        off += static_cast<int>(sizeof(csa::Barriers));
-        p.smem_bytes = off + 1024;
-        // More than half of the SM's shared memory: one CTA per SM, so the
-        // CTA's 512-column TMEM allocation never waits on a neighbour.
-        if (p.smem_bytes < kSmemLimit / 2 + 1024)
-            p.smem_bytes = kSmemLimit / 2 + 1024;
-        break;
-    }
-    if (p.stages < 2)
+    int off = 0;
+    p.off_q = off;
+    off += p.N * p.d * 2;
+    p.off_k = off;
+    int tail = 0;
+    tail += p.qps * p.H * 4;                                   // w
+    tail = (tail + 15) / 16 * 16;
+    tail += 2 * p.qps * static_cast<int>(sizeof(csa::QueryState));
+    p.wg_bytes = (static_cast<int>(sizeof(csa::WgScratch)) + 15) / 16 * 16;
+    tail += 2 * p.wg_bytes;
+    tail += (static_cast<int>(sizeof(csa::FinScratch)) + 15) / 16 * 16;
+    tail += static_cast<int>(sizeof(csa::Barriers)) + 16;
+    int stages = (kSmemLimit - 1024 - off - tail) / k_stage;
+    if (stages > csa::kMaxStages)
+        stages = csa::kMaxStages;
+    if (stages < 2)
         return CSA_ERR_UNSUPPORTED;
-    p.nqb = (p.S + p.qpb - 1) / p.qpb;
+    p.stages = stages;
+    off += stages * k_stage;
+    p.off_w = off;
+    off += p.qps * p.H * 4;
+    off = (off + 15) / 16 * 16;
+    p.off_state = off;
+    off += 2 * p.qps * static_cast<int>(sizeof(csa::QueryState));
+    p.off_wg = off;
+    off += 2 * p.wg_bytes;
+    p.off_fin = off;
+    off += (static_cast<int>(sizeof(csa::FinScratch)) + 15) / 16 * 16;
+    p.off_bar = off;
+    off += static_cast<int>(sizeof(csa::Barriers));
+    p.smem_bytes = off + 1024;
+    // More than half of the SM's shared memory: one CTA per SM, so the CTA's
+    // 512-column TMEM allocation never waits on a neighbour.
+    if (p.smem_bytes < kSmemLimit / 2 + 1024)
+        p.smem_bytes = kSmemLimit / 2 + 1024;
+    p.nqb = (p.S + p.qps - 1) / p.qps;
 
     // Key-range splits: only when there are too few query blocks to fill the
     // GPU; pick the count with the best last-wave occupancy.
@@ -252,7 +243,7 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
     plan.grid = p.n_items < sms ? p.n_items : sms;
     if (plan.grid < 1)
         plan.grid = 1;
-    plan.ws_cand = align256(static_cast<size_t>(plan.grid) * p.qpb * p.cap * 8);
+    plan.ws_cand = align256(static_cast<size_t>(plan.grid) * 2 * p.qps * p.cap * 8);
     plan.ws_part = nsplit > 1
                        ? align256(static_cast<size_t>(p.B) * p.S * nsplit * p.topk * 8)
                        : 0;
@@ -289,6 +280,7 @@ __global__ void pad_outputs_kernel(int32_t *idx, float *score, long long n)
 csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_t stream)
 {
     Params p = plan.p;
+    p.q = static_cast<const uint16_t *>(a->q);
     p.w = a->w;
     p.k_scale = a->k_scale;
     p.out_idx = a->out_idx;
@@ -373,7 +365,7 @@ csa_status_t csa_indexer_plan(const csa_args_t *args, csa_plan_t *out)
     out->threads = csa::kThreads;
     out->smem_bytes = plan.p.smem_bytes;
     out->stages = plan.p.stages;
-    out->queries_per_block = plan.p.qpb;
+    out->queries_per_block = plan.p.qps;
     out->num_splits = plan.p.nsplit;
     out->launches = plan.p.nsplit > 1 ? 2 : 1;
     out->workspace_bytes = plan.ws_total;
@@ -543,7 +535,7 @@ extern "C" csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStr
     // The per-CTA candidate lists scale with the grid: run fewer persistent
     // CTAs when a full grid's lists do not fit next to the split partials.
     if (plan.ws_total > kNoAllocScratchBytes) {
-        const size_t per_cta = static_cast<size_t>(plan.p.qpb) * plan.p.cap * 8;
+        const size_t per_cta = static_cast<size_t>(2) * plan.p.qps * plan.p.cap * 8;
         if (plan.ws_part + 256 > kNoAllocScratchBytes)
             return CSA_ERR_WORKSPACE;
         const size_t fit = (kNoAllocScratchBytes - plan.ws_part - 256) / per_cta;

@@ -8,6 +8,14 @@
 // "StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming Top-k",
 // abstract (top-k per query), with ties to the lower index.  Every real key is
 // non-zero, so 0 marks an empty slot.
+//
+// Two families of selection live here:
+//  * bucket selection (the fast path): scores are mapped monotonically onto
+//    NB buckets spanning the candidates' [min, max] score range, one shared
+//    histogram pass finds the bucket holding the k-th key, and a counting sort
+//    over buckets plus a tiny per-bucket sort orders the result;
+//  * radix selection over the 64-bit key (the exact fallback for degenerate
+//    ranges, e.g. many equal scores) and a bitonic sort.
 #pragma once
 #include <cstdint>
 
@@ -34,12 +42,13 @@ __device__ __forceinline__ uint64_t make_key(uint32_t ord, uint32_t s)
 }
 
 __device__ __forceinline__ int key_index(uint64_t k) { return static_cast<int>(~static_cast<uint32_t>(k)); }
-__device__ __forceinline__ float key_score(uint64_t k) { return score_of_ord(static_cast<uint32_t>(k >> 32)); }
+__device__ __forceinline__ uint32_t key_ord(uint64_t k) { return static_cast<uint32_t>(k >> 32); }
+__device__ __forceinline__ float key_score(uint64_t k) { return score_of_ord(key_ord(k)); }
 
-struct GroupScratch {
-    uint32_t hist[256];
-    int bcast[4];
-    int warp_sums[32];
+// Small per-group scratch for broadcasts and scans.
+struct GroupSmall {
+    int bcast[8];
+    uint32_t warp_sums[32];
 };
 
 __device__ __forceinline__ unsigned lanemask_lt()
@@ -66,7 +75,7 @@ __device__ __forceinline__ bool group_all(int bar, int nthreads, bool v)
 
 // Exclusive prefix sum of v over the group (thread order); *total = group sum.
 template <int NT>
-__device__ __forceinline__ int group_excl_scan(int v, GroupScratch *sc, int bar, int tid, int *total)
+__device__ __forceinline__ int group_excl_scan(int v, GroupSmall *gs, int bar, int tid, int *total)
 {
     const int lane = tid & 31, wid = tid >> 5;
     int x = v;
@@ -77,12 +86,12 @@ __device__ __forceinline__ int group_excl_scan(int v, GroupScratch *sc, int bar,
             x += y;
     }
     if (lane == 31)
-        sc->warp_sums[wid] = x;
+        gs->warp_sums[wid] = static_cast<uint32_t>(x);
     named_bar_sync(bar, NT);
     int base = 0, tot = 0;
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) {
-        const int s = sc->warp_sums[w];
+        const int s = static_cast<int>(gs->warp_sums[w]);
         base += w < wid ? s : 0;
         tot += s;
     }
@@ -91,14 +100,33 @@ __device__ __forceinline__ int group_excl_scan(int v, GroupScratch *sc, int bar,
     return base + x - v;
 }
 
+// Group-wide min of an unsigned value; every thread gets the result.
+template <int NT>
+__device__ __forceinline__ uint32_t group_min_u32(uint32_t v, GroupSmall *gs, int bar, int tid)
+{
+    const int lane = tid & 31, wid = tid >> 5;
+    const uint32_t m = __reduce_min_sync(0xffffffffu, v);
+    if (lane == 0)
+        gs->warp_sums[wid] = m;
+    named_bar_sync(bar, NT);
+    uint32_t r = 0xFFFFFFFFu;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w)
+        r = min(r, gs->warp_sums[w]);
+    named_bar_sync(bar, NT);
+    return r;
+}
+
+// ---------------------------------------------------------------------------- radix (exact)
+
 // Radix select over the group's keys (EPT per thread, 0 = empty), most
 // significant byte first.  Precondition: more than K non-zero keys, all
 // distinct.  Returns a bound L such that the number of keys >= L lies in
 // [K, K + slack] (exactly K when slack == 0); *kept = that number.  Every key
 // below L has at least K keys above it, so dropping it never loses a top-K key.
 template <int NT, int EPT>
-__device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, GroupScratch *sc,
-                                int bar, int tid, int *kept)
+__device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, uint32_t *hist,
+                                GroupSmall *gs, int bar, int tid, int *kept)
 {
     const int lane = tid & 31;
     uint64_t prefix = 0, mask = 0;
@@ -106,7 +134,7 @@ __device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, Grou
     int total_ge = 0;
     for (int pos = 56; pos >= 0; pos -= 8) {
         for (int i = tid; i < 256; i += NT)
-            sc->hist[i] = 0;
+            hist[i] = 0;
         named_bar_sync(bar, NT);
 #pragma unroll
         for (int i = 0; i < EPT; ++i) {
@@ -117,7 +145,7 @@ __device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, Grou
             if (match) {
                 const unsigned peers = __match_any_sync(act, digit);
                 if (lane == __ffs(peers) - 1)
-                    atomicAdd(&sc->hist[digit], static_cast<uint32_t>(__popc(peers)));
+                    atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(peers)));
             }
         }
         named_bar_sync(bar, NT);
@@ -126,10 +154,10 @@ __device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, Grou
             uint32_t sum = 0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                c[j] = sc->hist[lane * 8 + j];
+                c[j] = hist[lane * 8 + j];
                 sum += c[j];
             }
-            uint32_t suf = sum; // keys whose digit lies in this lane's bins or above
+            uint32_t suf = sum;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
@@ -143,9 +171,9 @@ __device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, Grou
 #pragma unroll
                 for (int j = 7; j >= 0; --j) {
                     if (above + c[j] >= nd) {
-                        sc->bcast[0] = lane * 8 + j;
-                        sc->bcast[1] = static_cast<int>(above);
-                        sc->bcast[2] = static_cast<int>(c[j]);
+                        gs->bcast[0] = lane * 8 + j;
+                        gs->bcast[1] = static_cast<int>(above);
+                        gs->bcast[2] = static_cast<int>(c[j]);
                         break;
                     }
                     above += c[j];
@@ -153,9 +181,10 @@ __device__ uint64_t radix_bound(const uint64_t (&e)[EPT], int K, int slack, Grou
             }
         }
         named_bar_sync(bar, NT);
-        const int digit = sc->bcast[0];
-        const int above = sc->bcast[1];
-        const int inb = sc->bcast[2];
+        const int digit = gs->bcast[0];
+        const int above = gs->bcast[1];
+        const int inb = gs->bcast[2];
+        named_bar_sync(bar, NT);
         need -= above;
         prefix |= static_cast<uint64_t>(digit) << pos;
         mask |= 0xFFull << pos;
@@ -173,8 +202,9 @@ __device__ void bitonic_sort_desc(uint64_t *a, int P, int bar, int tid)
 {
     for (int size = 2; size <= P; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const int sh = __ffs(stride) - 1;
             for (int p = tid; p < (P >> 1); p += NT) {
-                const int lo = 2 * stride * (p / stride) + (p % stride);
+                const int lo = ((p >> sh) << (sh + 1)) + (p & (stride - 1));
                 const int hi = lo + stride;
                 const bool desc = (lo & size) == 0;
                 const uint64_t x = a[lo], y = a[hi];
@@ -188,62 +218,137 @@ __device__ void bitonic_sort_desc(uint64_t *a, int P, int bar, int tid)
     }
 }
 
-// Shrinks the candidate list buf[0..n) (global memory, keys unique) to at
-// most K + slack keys that still contain the top K, in place.  Returns the
-// new length; *bound_ord receives the high word of the cut, so a later key
-// can only matter if its score's order image is >= *bound_ord.
+// Keeps the keys >= L of e[] (all non-zero keys when L == 1) at out[0..total)
+// in arbitrary order; returns total.  Also returns the smallest kept score
+// order image in *min_ord (0xFFFFFFFF when nothing is kept).
 template <int NT, int EPT>
-__device__ int compact_candidates(uint64_t *buf, int n, int K, int slack, GroupScratch *sc, int bar,
-                                  int tid, uint32_t *bound_ord)
+__device__ int write_kept(const uint64_t (&e)[EPT], uint64_t L, uint64_t *out, GroupSmall *gs,
+                          int bar, int tid, uint32_t *min_ord)
 {
-    uint64_t e[EPT];
+    int mine = 0;
+    uint32_t mn = 0xFFFFFFFFu;
 #pragma unroll
     for (int i = 0; i < EPT; ++i) {
-        const int j = i * NT + tid;
-        e[i] = j < n ? buf[j] : 0ull;
+        const bool keep = e[i] != 0 && e[i] >= L;
+        mine += keep ? 1 : 0;
+        mn = keep ? min(mn, key_ord(e[i])) : mn;
     }
-    int kept;
-    const uint64_t L = radix_bound<NT, EPT>(e, K, slack, sc, bar, tid, &kept);
-    int mine = 0;
-#pragma unroll
-    for (int i = 0; i < EPT; ++i)
-        mine += (e[i] != 0 && e[i] >= L) ? 1 : 0;
     int total;
-    int off = group_excl_scan<NT>(mine, sc, bar, tid, &total);
-#pragma unroll
-    for (int i = 0; i < EPT; ++i)
-        if (e[i] != 0 && e[i] >= L)
-            buf[off++] = e[i];
-    *bound_ord = static_cast<uint32_t>(L >> 32);
-    named_bar_sync(bar, NT); // writes visible to the whole group before reuse
-    return total;
-}
-
-// Exact selection of the min(K, #non-zero) largest keys among e[] into
-// out[0..kept) (shared memory, unordered), zero-filled up to `pad_to`.
-template <int NT, int EPT>
-__device__ int select_topk(const uint64_t (&e)[EPT], int n, int K, uint64_t *out, int pad_to,
-                           GroupScratch *sc, int bar, int tid)
-{
-    uint64_t L = 1;
-    int kept = n;
-    if (n > K) {
-        L = radix_bound<NT, EPT>(e, K, 0, sc, bar, tid, &kept);
-    }
-    int mine = 0;
-#pragma unroll
-    for (int i = 0; i < EPT; ++i)
-        mine += (e[i] != 0 && e[i] >= L) ? 1 : 0;
-    int total;
-    int off = group_excl_scan<NT>(mine, sc, bar, tid, &total);
+    int off = group_excl_scan<NT>(mine, gs, bar, tid, &total);
 #pragma unroll
     for (int i = 0; i < EPT; ++i)
         if (e[i] != 0 && e[i] >= L)
             out[off++] = e[i];
-    for (int i = total + tid; i < pad_to; i += NT)
-        out[i] = 0ull;
-    named_bar_sync(bar, NT);
+    *min_ord = group_min_u32<NT>(mn, gs, bar, tid);
     return total;
+}
+
+// ---------------------------------------------------------------------------- buckets
+
+// Monotone map of scores in [lo, hi] onto buckets [0, NB): b(x) never
+// decreases when x increases (fp32 subtraction, multiplication by a positive
+// constant and truncation are all monotone), so bucket order is score order.
+struct BucketMap {
+    float lo, inv;
+    bool ok;
+};
+
+__device__ __forceinline__ BucketMap bucket_map(uint32_t min_ord, uint32_t max_ord, int NB)
+{
+    BucketMap m;
+    const float lo = score_of_ord(min_ord);
+    const float hi = score_of_ord(max_ord);
+    const float span = hi - lo;
+    m.lo = lo;
+    m.inv = static_cast<float>(NB) / span;
+    m.ok = max_ord > min_ord && span > 0.0f && isfinite(span) && isfinite(m.inv) && isfinite(lo);
+    return m;
+}
+
+__device__ __forceinline__ int bucket_of(float s, const BucketMap &m, int NB)
+{
+    const float x = (s - m.lo) * m.inv;
+    int b = static_cast<int>(x);
+    b = b < 0 ? 0 : b;
+    return b > NB - 1 ? NB - 1 : b;
+}
+
+// After a histogram hist[0..NB) of the group's keys, find the bucket b* that
+// holds the need-th largest key: above(b*) < need <= above(b*) + hist[b*],
+// where above(b) counts keys in buckets > b.  gs->bcast = {b*, above(b*),
+// hist[b*], largest bucket count among buckets >= b*}.  With write_above,
+// hist[b] is replaced by above(b) (the first output slot of bucket b when
+// buckets are laid out from the highest down).  Precondition: at least
+// `need` keys in the histogram.
+template <int NT, int NB>
+__device__ void bucket_boundary(uint32_t *hist, int need, bool write_above, GroupSmall *gs, int bar,
+                                int tid)
+{
+    constexpr int PER = NB / NT;
+    const int lane = tid & 31, wid = tid >> 5;
+    uint32_t c[PER];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        c[j] = hist[tid * PER + j];
+        sum += c[j];
+    }
+    uint32_t suf = sum; // inclusive suffix over threads within the warp
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 32)
+            suf += t;
+    }
+    if (lane == 0)
+        gs->warp_sums[wid] = suf; // the warp's total
+    named_bar_sync(bar, NT);
+    uint32_t higher = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w)
+        higher += w > wid ? gs->warp_sums[w] : 0u;
+    suf += higher;
+    const uint32_t above_thread = suf - sum;
+    const uint32_t nd = static_cast<uint32_t>(need);
+    if (write_above) {
+        uint32_t run = above_thread;
+#pragma unroll
+        for (int j = PER - 1; j >= 0; --j) {
+            hist[tid * PER + j] = run;
+            run += c[j];
+        }
+    }
+    if (above_thread < nd && nd <= suf) {
+        uint32_t above = above_thread;
+#pragma unroll
+        for (int j = PER - 1; j >= 0; --j) {
+            if (above + c[j] >= nd) {
+                gs->bcast[0] = tid * PER + j;
+                gs->bcast[1] = static_cast<int>(above);
+                gs->bcast[2] = static_cast<int>(c[j]);
+                break;
+            }
+            above += c[j];
+        }
+    }
+    named_bar_sync(bar, NT);
+    // largest bucket at or above b*
+    const int bstar = gs->bcast[0];
+    uint32_t mx = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+        mx = (tid * PER + j >= bstar) ? max(mx, c[j]) : mx;
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0)
+        gs->warp_sums[wid] = mx;
+    named_bar_sync(bar, NT);
+    if (tid == 0) {
+        uint32_t m = 0;
+        for (int w = 0; w < NT / 32; ++w)
+            m = max(m, gs->warp_sums[w]);
+        gs->bcast[3] = static_cast<int>(m);
+    }
+    named_bar_sync(bar, NT);
 }
 
 __host__ __device__ constexpr int pow2_at_least(int x)
