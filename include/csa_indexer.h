@@ -122,10 +122,13 @@ csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
  * the library holds until the process exits.  The caller still passes all
  * inputs and outputs.  The first call on each device looks up that array's
  * device address (cudaGetSymbolAddress); make that first call before any
- * stream capture.  If a full grid's scratch does not fit, the call runs fewer
- * persistent CTAs; if the shape needs more than the array even then (large
- * B*S*topk with key-range splits), it returns CSA_ERR_WORKSPACE and launches
- * nothing.  All calls share the one array and nothing in it needs to start at
+ * stream capture.  The scratch holds the candidate lists of the queries in
+ * flight (B * queries-per-block * splits lists of about 2*topk 8-byte keys per
+ * block of queries); when all of them do not fit, the call runs as several
+ * launch chunks of query blocks.  If one query block of every sequence already
+ * needs more than the array (very large B * topk), it returns
+ * CSA_ERR_WORKSPACE and launches nothing.  All calls share the one array and
+ * nothing in it needs to start at
  * zero, but two calls that overlap on the GPU (different streams, or
  * different host threads) race on it and give undefined results: serialise
  * them.

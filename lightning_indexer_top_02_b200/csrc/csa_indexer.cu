@@ -1,7 +1,8 @@
 // csa_indexer.cu -- host side of the C ABI declared in include/csa_indexer.h:
-// argument validation, work planning (query blocks, sub-blocks, key splits,
-// pipeline depth, candidate capacity), TMA descriptors, workspace layout and
-// launches of the fused indexer/top-k kernel and the split merge.
+// argument validation, work planning (query blocks, key splits, pipeline
+// depth, candidate capacity, launch chunks), TMA descriptors, workspace layout
+// and the launches: per chunk of query blocks, the fused scoring/filter kernel
+// and then the exact top-k selection over its candidate lists.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,6 +13,7 @@
 
 #include "csa_indexer.h"
 #include "indexer_kernel.cuh"
+#include "select_kernel.cuh"
 
 namespace {
 
@@ -57,10 +59,18 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Workspace the default entry points may use for one launch chunk; larger
+// problems run as several chunks of query blocks.
+constexpr size_t kDefaultWorkspaceCap = size_t(16) << 30;
+
 struct Plan {
-    Params p;
+    Params p;          // qb_lo, nqb and n_items describe the first chunk
     int grid;
-    size_t ws_cand, ws_part, ws_total;
+    int nqb_total;     // query blocks per batch
+    int qb_chunk;      // query blocks per batch in one launch chunk
+    int chunks;
+    int fast_fc, fast_fq; // epilogue fast path (0 = generic)
+    size_t ws_lists, ws_counts, ws_total;
 };
 
 csa_status_t validate(const csa_args_t *a)
@@ -125,7 +135,7 @@ int max_tiles(const csa_args_t *a, long long q_offset)
     return static_cast<int>((nvis + csa::kTileKeys - 1) / csa::kTileKeys);
 }
 
-csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
+csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
 {
     Params p;
     std::memset(&p, 0, sizeof p);
@@ -176,10 +186,9 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
     int tail = 0;
     tail += p.qps * p.H * 4;                                   // w
     tail = (tail + 15) / 16 * 16;
-    tail += 2 * p.qps * static_cast<int>(sizeof(csa::QueryState));
+    tail += p.qps * static_cast<int>(sizeof(csa::QueryState));
     p.wg_bytes = (static_cast<int>(sizeof(csa::WgScratch)) + 15) / 16 * 16;
     tail += 2 * p.wg_bytes;
-    tail += (static_cast<int>(sizeof(csa::FinScratch)) + 15) / 16 * 16;
     tail += static_cast<int>(sizeof(csa::Barriers)) + 16;
     int stages = (kSmemLimit - 1024 - off - tail) / k_stage;
     if (stages > csa::kMaxStages)
@@ -192,11 +201,10 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
     off += p.qps * p.H * 4;
     off = (off + 15) / 16 * 16;
     p.off_state = off;
-    off += 2 * p.qps * static_cast<int>(sizeof(csa::QueryState));
+    off += p.qps * static_cast<int>(sizeof(csa::QueryState));
+    off = (off + 15) / 16 * 16;
     p.off_wg = off;
     off += 2 * p.wg_bytes;
-    p.off_fin = off;
-    off += (static_cast<int>(sizeof(csa::FinScratch)) + 15) / 16 * 16;
     p.off_bar = off;
     off += static_cast<int>(sizeof(csa::Barriers));
     p.smem_bytes = off + 1024;
@@ -204,19 +212,17 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
     // 512-column TMEM allocation never waits on a neighbour.
     if (p.smem_bytes < kSmemLimit / 2 + 1024)
         p.smem_bytes = kSmemLimit / 2 + 1024;
-    p.nqb = (p.S + p.qps - 1) / p.qps;
+    const int nqb_total = (p.S + p.qps - 1) / p.qps;
 
     // Key-range splits: only when there are too few query blocks to fill the
     // GPU; pick the count with the best last-wave occupancy.
-    const long long items_base = static_cast<long long>(p.B) * p.nqb;
+    const long long items_base = static_cast<long long>(p.B) * nqb_total;
     int nsplit = 1;
     if (a->num_splits > 0) {
         nsplit = a->num_splits;
     } else if (items_base < 4ll * sms) {
         const int tiles = max_tiles(a, p.q_offset);
-        int max_split = 8192 / p.topk;
-        if (max_split > 16)
-            max_split = 16;
+        int max_split = 16;
         if (max_split > tiles)
             max_split = tiles;
         double best = -1.0;
@@ -231,23 +237,44 @@ csa_status_t make_plan(const csa_args_t *a, int sms, Plan *out)
             }
         }
     }
-    if (nsplit < 1 || static_cast<long long>(nsplit) * p.topk > 8192)
+    if (nsplit < 1 || nsplit > csa::kSelMaxSplits)
         return CSA_ERR_UNSUPPORTED;
     p.nsplit = nsplit;
-    const long long items = items_base * nsplit;
-    if (items >= (1ll << 31))
+
+    // Candidate lists: one per (query, split), cap keys each, plus its length.
+    // A launch chunk covers qb_chunk query blocks of every batch.
+    const size_t rows_per_qb = static_cast<size_t>(p.B) * p.qps;
+    const size_t lists_per_qb = rows_per_qb * nsplit * p.cap * 8;
+    const size_t counts_per_qb = rows_per_qb * nsplit * 4;
+    const size_t per_qb = lists_per_qb + counts_per_qb;
+    long long qb_chunk = nqb_total;
+    if (ws_cap < 512 + per_qb)
+        return CSA_ERR_WORKSPACE;
+    if (static_cast<size_t>(qb_chunk) * per_qb + 512 > ws_cap)
+        qb_chunk = static_cast<long long>((ws_cap - 512) / per_qb);
+    if (qb_chunk < 1)
+        return CSA_ERR_WORKSPACE;
+    const long long items = static_cast<long long>(p.B) * qb_chunk * nsplit;
+    if (items >= (1ll << 31) || static_cast<long long>(p.B) * qb_chunk * p.qps >= (1ll << 31))
         return CSA_ERR_UNSUPPORTED;
+    p.qb_lo = 0;
+    p.nqb = static_cast<int>(qb_chunk);
     p.n_items = static_cast<int>(items);
 
     Plan plan;
+    plan.nqb_total = nqb_total;
+    plan.qb_chunk = static_cast<int>(qb_chunk);
+    plan.chunks = static_cast<int>((nqb_total + qb_chunk - 1) / qb_chunk);
     plan.grid = p.n_items < sms ? p.n_items : sms;
     if (plan.grid < 1)
         plan.grid = 1;
-    plan.ws_cand = align256(static_cast<size_t>(plan.grid) * 2 * p.qps * p.cap * 8);
-    plan.ws_part = nsplit > 1
-                       ? align256(static_cast<size_t>(p.B) * p.S * nsplit * p.topk * 8)
-                       : 0;
-    plan.ws_total = plan.ws_cand + plan.ws_part;
+    plan.ws_lists = align256(static_cast<size_t>(qb_chunk) * lists_per_qb);
+    plan.ws_counts = align256(static_cast<size_t>(qb_chunk) * counts_per_qb);
+    plan.ws_total = plan.ws_lists + plan.ws_counts;
+    // Epilogue fast path: whole 32-column queries, 64 or 128 columns per group.
+    const int cols = p.qpw * p.H;
+    plan.fast_fc = (p.H >= 32 && (cols == 64 || cols == 128)) ? cols : 0;
+    plan.fast_fq = plan.fast_fc ? p.qpw : 0;
     plan.p = p;
     *out = plan;
     return CSA_OK;
@@ -277,17 +304,30 @@ __global__ void pad_outputs_kernel(int32_t *idx, float *score, long long n)
     }
 }
 
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
+
+KernelFn pick_kernel(const Plan &plan)
+{
+    switch (plan.fast_fc * 8 + plan.fast_fq) {
+    case 64 * 8 + 1: return csa::indexer_topk_kernel<64, 1, true>;
+    case 64 * 8 + 2: return csa::indexer_topk_kernel<64, 2, true>;
+    case 128 * 8 + 1: return csa::indexer_topk_kernel<128, 1, true>;
+    case 128 * 8 + 2: return csa::indexer_topk_kernel<128, 2, true>;
+    case 128 * 8 + 4: return csa::indexer_topk_kernel<128, 4, true>;
+    default: break;
+    }
+    return plan.p.H >= 32 ? csa::indexer_topk_kernel<0, 0, true>
+                          : csa::indexer_topk_kernel<0, 0, false>;
+}
+
 csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_t stream)
 {
     Params p = plan.p;
     p.q = static_cast<const uint16_t *>(a->q);
     p.w = a->w;
     p.k_scale = a->k_scale;
-    p.out_idx = a->out_idx;
-    p.out_score = a->out_score;
-    p.cand = reinterpret_cast<uint64_t *>(ws);
-    p.part = plan.ws_part ? reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(ws) + plan.ws_cand)
-                          : nullptr;
+    p.lists = reinterpret_cast<uint64_t *>(ws);
+    p.counts = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + plan.ws_lists);
     p.wait_limit = static_cast<long long>(g_wait_limit);
 
     CUtensorMap tmQ, tmK;
@@ -301,20 +341,41 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
                    csa::kTileKeys, swz))
         return CSA_ERR_CUDA;
 
-    const bool ge32 = p.H >= 32;
-    auto kern = ge32 ? csa::indexer_topk_kernel<true> : csa::indexer_topk_kernel<false>;
+    const KernelFn kern = pick_kernel(plan);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes) !=
         cudaSuccess)
         return CSA_ERR_CUDA;
-    kern<<<plan.grid, csa::kThreads, p.smem_bytes, stream>>>(tmQ, tmK, p);
-    if (cudaGetLastError() != cudaSuccess)
+    const int sel_smem = static_cast<int>(sizeof(csa::SelSmem)) + 16;
+    if (cudaFuncSetAttribute(csa::select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sel_smem) != cudaSuccess)
         return CSA_ERR_CUDA;
-    if (p.nsplit > 1) {
-        const int rows = p.B * p.S;
-        const int sms = device_sms();
-        int grid = rows < sms * 8 ? rows : sms * 8;
-        csa::merge_splits_kernel<<<grid, csa::kMergeThreads, 0, stream>>>(
-            p.part, rows, p.nsplit, p.topk, p.out_idx, p.out_score);
+    const int sms = device_sms();
+    for (int qb_lo = 0; qb_lo < plan.nqb_total; qb_lo += plan.qb_chunk) {
+        const int nqb = plan.nqb_total - qb_lo < plan.qb_chunk ? plan.nqb_total - qb_lo
+                                                              : plan.qb_chunk;
+        p.qb_lo = qb_lo;
+        p.nqb = nqb;
+        p.n_items = p.B * nqb * p.nsplit;
+        const int grid = p.n_items < plan.grid ? p.n_items : plan.grid;
+        kern<<<grid, csa::kThreads, p.smem_bytes, stream>>>(tmQ, tmK, p);
+        if (cudaGetLastError() != cudaSuccess)
+            return CSA_ERR_CUDA;
+        csa::SelParams sp;
+        sp.lists = p.lists;
+        sp.counts = p.counts;
+        sp.rows = p.B * nqb * p.qps;
+        sp.nsplit = p.nsplit;
+        sp.cap = p.cap;
+        sp.topk = p.topk;
+        sp.B = p.B;
+        sp.S = p.S;
+        sp.qps = p.qps;
+        sp.nqb = nqb;
+        sp.qb_lo = qb_lo;
+        sp.out_idx = a->out_idx;
+        sp.out_score = a->out_score;
+        const int sel_grid = sp.rows < 3 * sms ? sp.rows : 3 * sms;
+        csa::select_topk_kernel<<<sel_grid, csa::kSelThreads, sel_smem, stream>>>(sp);
         if (cudaGetLastError() != cudaSuccess)
             return CSA_ERR_CUDA;
     }
@@ -335,7 +396,7 @@ size_t csa_indexer_workspace_size(const csa_args_t *args)
     if (sms <= 0)
         return 0;
     Plan plan;
-    if (make_plan(args, sms, &plan) != CSA_OK)
+    if (make_plan(args, sms, kDefaultWorkspaceCap, &plan) != CSA_OK)
         return 0;
     return plan.ws_total;
 }
@@ -358,7 +419,7 @@ csa_status_t csa_indexer_plan(const csa_args_t *args, csa_plan_t *out)
     if (sms <= 0)
         return CSA_ERR_CUDA;
     Plan plan;
-    st = make_plan(args, sms, &plan);
+    st = make_plan(args, sms, kDefaultWorkspaceCap, &plan);
     if (st != CSA_OK)
         return st;
     out->grid = plan.grid;
@@ -367,7 +428,7 @@ csa_status_t csa_indexer_plan(const csa_args_t *args, csa_plan_t *out)
     out->stages = plan.p.stages;
     out->queries_per_block = plan.p.qps;
     out->num_splits = plan.p.nsplit;
-    out->launches = plan.p.nsplit > 1 ? 2 : 1;
+    out->launches = 2 * plan.chunks;
     out->workspace_bytes = plan.ws_total;
     return CSA_OK;
 }
@@ -390,7 +451,7 @@ csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace, size_t
     if (sms <= 0)
         return CSA_ERR_CUDA;
     Plan plan;
-    st = make_plan(args, sms, &plan);
+    st = make_plan(args, sms, kDefaultWorkspaceCap, &plan);
     if (st != CSA_OK)
         return st;
     if (workspace) {
@@ -528,28 +589,32 @@ extern "C" csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStr
     const int sms = device_sms();
     if (sms <= 0)
         return CSA_ERR_CUDA;
+    // The candidate lists scale with the number of query blocks in flight:
+    // the plan runs as many launch chunks as the fixed scratch requires.
     Plan plan;
-    st = make_plan(args, sms, &plan);
+    st = make_plan(args, sms, kNoAllocScratchBytes, &plan);
     if (st != CSA_OK)
         return st;
-    // The per-CTA candidate lists scale with the grid: run fewer persistent
-    // CTAs when a full grid's lists do not fit next to the split partials.
-    if (plan.ws_total > kNoAllocScratchBytes) {
-        const size_t per_cta = static_cast<size_t>(2) * plan.p.qps * plan.p.cap * 8;
-        if (plan.ws_part + 256 > kNoAllocScratchBytes)
-            return CSA_ERR_WORKSPACE;
-        const size_t fit = (kNoAllocScratchBytes - plan.ws_part - 256) / per_cta;
-        if (fit < 1)
-            return CSA_ERR_WORKSPACE;
-        plan.grid = static_cast<int>(fit < static_cast<size_t>(plan.grid) ? fit : plan.grid);
-        plan.ws_cand = align256(static_cast<size_t>(plan.grid) * per_cta);
-        plan.ws_total = plan.ws_cand + plan.ws_part;
-        if (plan.ws_total > kNoAllocScratchBytes)
-            return CSA_ERR_WORKSPACE;
-    }
     void *scratch = nullptr;
     st = noalloc_scratch(&scratch);
     if (st != CSA_OK)
         return st;
     return launch(args, plan, scratch, stream);
 }
+
+#ifdef CSA_PROFILE
+// Profiling build only: per-CTA role counters of the last launches.
+extern "C" int csa_profile_read(unsigned long long *out, int n)
+{
+    const size_t bytes = sizeof(unsigned long long) * csa::kProfCtas * 32;
+    if (n * sizeof(unsigned long long) < bytes)
+        return -1;
+    return cudaMemcpyFromSymbol(out, csa::g_csa_prof, bytes) == cudaSuccess ? 0 : -1;
+}
+
+extern "C" int csa_profile_reset(void)
+{
+    static unsigned long long zero[csa::kProfCtas][32];
+    return cudaMemcpyToSymbol(csa::g_csa_prof, zero, sizeof zero) == cudaSuccess ? 0 : -1;
+}
+#endif

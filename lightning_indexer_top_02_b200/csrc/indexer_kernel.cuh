@@ -1,30 +1,37 @@
-// indexer_kernel.cuh -- the fused lightning-indexer + streaming top-k kernel.
+// indexer_kernel.cuh -- the fused lightning-indexer scoring + streaming
+// candidate filter.
 //
 // One persistent CTA per SM walks work items (batch b, block of qps queries,
 // range of key tiles).  For each 128-key tile the tensor cores compute the
 // logits L[s, (t,h)] = k[s,:] . q[t,h,:] for every head of the item's queries
 // ("StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
 // Top-k", abstract: the lightning indexer scores compressed keys per query),
-// with keys as the MMA's M dimension so that each TMEM lane -- one epilogue
-// thread -- holds one key's logits for every (query, head).  The epilogue
-// applies ReLU and the head weights without leaving the thread, masks keys the
-// query may not see, and streams the surviving (score, index) pairs into a
-// per-query candidate list that is cut back to the top k plus slack whenever
-// it could overflow.  When an item's key range is done, a separate warpgroup
-// reduces each list to the exact top k and sorts it while the next item's
-// tiles already flow through the tensor cores, so the [B,S,H_I,T] score tensor
-// never exists and the selection stays off the MMA's critical path.
+// with keys as the MMA's M dimension so that each TMEM lane holds one key's
+// logits for every (query, head).  The epilogue applies ReLU and the head
+// weights, masks keys the query may not see, and streams the surviving
+// (score, index) pairs into the query's candidate list in global memory; a
+// list that could overflow is cut back in place to the top k plus slack and
+// the admission bound rises to the smallest score kept.  When an item's key
+// range is done the list holds a superset of the query's top k over that
+// range; select_kernel.cuh turns the lists into the exact, sorted top k.  The
+// [B,S,H_I,T] score tensor never exists and the extra memory is O(S * k).
 //
-// Warp roles (448 threads):
-//   warp 0       TMA producer: the query block once per item (with an L2
-//                prefetch of the next item's), key tiles into a ring
-//   warp 1       TMEM owner and MMA issuer (one thread): per key tile, d/16
-//                tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
-//                256-column TMEM accumulators
-//   warps 2..5   epilogue warpgroup 0: the first half of the item's queries
-//   warps 6..9   epilogue warpgroup 1: the second half (idle when qps == 1)
-//   warps 10..13 finalizer: exact top-k + sort of each finished query, from
-//                double-buffered candidate lists
+// Warp roles (320 threads):
+//   warp 0      TMA producer: the query block once per item (with an L2
+//               prefetch of the next item's), key tiles into a ring
+//   warp 1      TMEM owner and MMA issuer (one thread): per key tile, d/16
+//               tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
+//               256-column TMEM accumulators
+//   warps 2..5  epilogue warpgroup 0: the first half of the item's queries
+//   warps 6..9  epilogue warpgroup 1: the second half (idle when qps == 1)
+//
+// Epilogue fast path (H_I >= 32, at most 128 TMEM columns per warpgroup): a
+// warp reads its 32 TMEM lanes with two 16-lane x 256-bit loads, so every
+// thread sees a fixed quarter of the columns of four keys; the head weights of
+// that quarter stay in registers for the whole item, the accumulator slot is
+// handed back to the MMA as soon as the loads land, and two butterfly shuffles
+// leave each thread with one key's complete scores.  Other shapes read one key
+// per thread with 32-lane loads and weights from shared memory.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -36,18 +43,71 @@ namespace csa {
 
 constexpr int kTileKeys = 128;   // MMA M: keys per tile
 constexpr int kSlotCols = 256;   // TMEM columns per accumulator slot
-constexpr int kThreads = 448;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kGroupThreads = 128;
-constexpr int kBarWg0 = 1, kBarWg1 = 2, kBarFin = 3;  // named barriers
+constexpr int kBarWg0 = 1, kBarWg1 = 2;  // named barriers of the epilogue warpgroups
 constexpr int kEpt = 32;         // candidate keys per thread in a group (cap <= 4096)
 constexpr int kMaxStages = 8;
 constexpr int kMaxTopk = 2048;
 constexpr int kNbCompact = 1024; // buckets of the compaction histogram
-constexpr int kNbFinal = 1024;   // buckets of the final selection histogram
-constexpr int kGatherMax = 128;  // keys of the boundary bucket resolved in place
-constexpr int kBucketSortMax = 32; // larger buckets take the exact fallback
 
-enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleFinal = 4 };
+enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelect = 4 };
+
+// Optional per-role cycle counters (built only with -DCSA_PROFILE): where each
+// role spends its time, recorded by one thread per role and CTA.
+enum ProfSlot : int {
+    kPfProdQEmpty, kPfProdKEmpty, kPfMmaQFull, kPfMmaKFull, kPfMmaAccEmpty, kPfMmaTotal,
+    kPfEpiAccFull, kPfEpiCompact, kPfEpiTotal, kPfEpiCompactCount, kPfEpiTiles, kPfEpiMath,
+    kPfEpiTileBar, kPfSlots
+};
+#ifdef CSA_PROFILE
+constexpr int kProfCtas = 160;
+__device__ unsigned long long g_csa_prof[kProfCtas][32];
+
+struct ProfAcc {
+    unsigned long long v[kPfSlots];
+    __device__ __forceinline__ ProfAcc()
+    {
+#pragma unroll
+        for (int i = 0; i < kPfSlots; ++i)
+            v[i] = 0;
+    }
+    __device__ __forceinline__ void flush(bool rec)
+    {
+        if (rec && blockIdx.x < kProfCtas) {
+#pragma unroll
+            for (int i = 0; i < kPfSlots; ++i)
+                if (v[i])
+                    atomicAdd(&g_csa_prof[blockIdx.x][i], v[i]);
+        }
+    }
+};
+
+struct Prof {
+    long long t0;
+    __device__ __forceinline__ void start() { t0 = clock64(); }
+    __device__ __forceinline__ void add(ProfAcc &a, int slot, bool rec)
+    {
+        if (rec)
+            a.v[slot] += static_cast<unsigned long long>(clock64() - t0);
+    }
+    __device__ __forceinline__ void count(ProfAcc &a, int slot, bool rec)
+    {
+        if (rec)
+            a.v[slot] += 1;
+    }
+};
+#else
+struct ProfAcc {
+    __device__ __forceinline__ void flush(bool) {}
+};
+struct Prof {
+    __device__ __forceinline__ void start() {}
+    __device__ __forceinline__ void add(ProfAcc &, int, bool) {}
+    __device__ __forceinline__ void count(ProfAcc &, int, bool) {}
+};
+#endif
 
 struct Params {
     int B, S, T, H, d, m, topk, causal, mode, key_fp8;
@@ -56,29 +116,30 @@ struct Params {
     int N;        // MMA N = qps * H (<= 256)
     int n_wg;     // epilogue warpgroups in use (1 or 2)
     int qpw;      // queries per epilogue warpgroup = qps / n_wg
-    int nqb;      // query blocks per batch
+    int qb_lo;    // first query block (per batch) of this launch
+    int nqb;      // query blocks per batch in this launch
     int nsplit;   // key-range splits per query block
     int n_items;
     int stages;
-    int cap;      // candidate list capacity per query
+    int cap;      // candidate list capacity per query and split
     int slack;    // compaction keeps at most topk + slack when it must cut exactly
     int row_bytes;   // bytes of one swizzled operand row: min(128, 2*d)
     int n_chunks;    // d*2 / row_bytes
     // shared memory carve-up (byte offsets from the 1024-aligned base)
-    int off_q, off_k, off_w, off_state, off_wg, off_fin, off_bar, smem_bytes;
+    int off_q, off_k, off_w, off_state, off_wg, off_bar, smem_bytes;
     int wg_bytes;    // per-warpgroup scratch
     const uint16_t *q; // only for L2 prefetch; loads go through the tensor map
     const float *w;
     const float *k_scale;
-    int32_t *out_idx;
-    float *out_score;
-    uint64_t *cand;  // [gridDim.x][2][qps][cap]
-    uint64_t *part;  // [B*S][nsplit][topk] (nsplit > 1)
+    uint64_t *lists; // [list row][nsplit][cap] candidate keys
+    int *counts;     // [list row][nsplit] keys in each list
     long long wait_limit;
 };
 
+// List row of query j of query block qb (relative to qb_lo) in batch b:
+// (b * nqb + qb) * qps + j.
 struct Item {
-    int b, q0, nq, tile_begin, tile_end, split;
+    int b, q0, nq, tile_begin, tile_end, split, lrow;
 };
 
 __device__ __forceinline__ int visible_count(const Params &p, long long t)
@@ -100,9 +161,10 @@ __device__ __forceinline__ Item decode_item(const Params &p, int id)
     it.split = id % p.nsplit;
     const int r = id / p.nsplit;
     it.b = r % p.B;
-    const int qb = p.nqb - 1 - r / p.B;
-    it.q0 = qb * p.qps;
+    const int qbr = p.nqb - 1 - r / p.B;
+    it.q0 = (p.qb_lo + qbr) * p.qps;
     it.nq = min(p.qps, p.S - it.q0);
+    it.lrow = (it.b * p.nqb + qbr) * p.qps;
     const int nvis = visible_count(p, static_cast<long long>(it.q0 + it.nq - 1) + p.q_offset);
     const int nkt = (nvis + kTileKeys - 1) / kTileKeys;
     it.tile_begin = static_cast<int>(static_cast<long long>(it.split) * nkt / p.nsplit);
@@ -114,19 +176,16 @@ struct Barriers {
     uint64_t q_full, q_empty, drain, pad0;
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t acc_full[2], acc_empty[2];
-    uint64_t fin_full[2], fin_empty[2];
     uint32_t tmem_addr;
     int abort;
 };
 
-// Per-query streaming state (double-buffered by item parity).
+// Per-query streaming state of the current item.
 struct QueryState {
     int cnt;          // candidates in the list
     uint32_t bound;   // admit a key only if ord(score) >= bound
-    uint32_t min_ord; // smallest / largest score order image in the list
-    uint32_t max_ord;
     int vis_end;      // keys s < vis_end are visible to this query
-    int pad[3];
+    int pad;
 };
 
 // Bounded wait used when unwinding: ignores the abort flag and the (possibly
@@ -157,12 +216,16 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
                              uint8_t *smem, Barriers *bars, const WaitCtl &ctl)
 {
     int kload = 0, qload = 0;
+    ProfAcc pa;
+    Prof pf;
     const uint32_t q_bytes = static_cast<uint32_t>(p.N * p.d * 2);
     const uint32_t k_bytes = static_cast<uint32_t>(kTileKeys * p.d * 2);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
+        pf.start();
         if (!wait_bounded(&bars->q_empty, (qload & 1) ^ 1, ctl, kRoleProducer, id))
             goto unwind;
+        pf.add(pa, kPfProdQEmpty, true);
         const size_t wrow = static_cast<size_t>(it.b) * p.S + it.q0;
         if (it.tile_end > it.tile_begin) {
             mbar_arrive_expect_tx(&bars->q_full, q_bytes);
@@ -187,9 +250,11 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
         }
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
             const int stage = kload % p.stages;
+            pf.start();
             if (!wait_bounded(&bars->k_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
                               kRoleProducer, id))
                 goto unwind;
+            pf.add(pa, kPfProdKEmpty, true);
             mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
             uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
             const int row = it.b * p.T + t * kTileKeys;
@@ -209,6 +274,7 @@ unwind:
     }
     if (qload > 0)
         wait_drain(&bars->q_full, (qload - 1) & 1);
+    pa.flush(true);
 }
 
 // ------------------------------------------------------------------ MMA issuer
@@ -216,22 +282,31 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
                         const WaitCtl &ctl)
 {
     int kuse = 0, quse = 0, acc_use = 0;
-    const uint32_t idesc = instr_desc_f16(p.N, p.key_fp8 ? 0 : 1);
+    ProfAcc pa;
+    Prof pf, pt;
+    pt.start();
+    const uint32_t idesc = instr_desc_f16(p.N, 1);
     const int ksteps_per_chunk = p.row_bytes / 32;  // 16 elements (32 B) per MMA K step
     const uint32_t q_base = smem_u32(smem + p.off_q);
     const uint32_t k_base = smem_u32(smem + p.off_k);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
+        pf.start();
         if (!wait_bounded(&bars->q_full, quse & 1, ctl, kRoleMma, id))
             goto unwind;
+        pf.add(pa, kPfMmaQFull, true);
         tc_fence_after();
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
             const int stage = kuse % p.stages;
+            pf.start();
             if (!wait_bounded(&bars->k_full[stage], (kuse / p.stages) & 1, ctl, kRoleMma, id))
                 goto unwind;
+            pf.add(pa, kPfMmaKFull, true);
             const int slot = acc_use & 1;
+            pf.start();
             if (!wait_bounded(&bars->acc_empty[slot], ((acc_use >> 1) & 1) ^ 1, ctl, kRoleMma, id))
                 goto unwind;
+            pf.add(pa, kPfMmaAccEmpty, true);
             tc_fence_after();
             const uint32_t a_tile = k_base + stage * kTileKeys * p.d * 2;
             const uint32_t d_tmem = tmem_base + slot * kSlotCols;
@@ -256,8 +331,10 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
         ++quse;
     }
 unwind:
+    pt.add(pa, kPfMmaTotal, true);
     mma_commit(&bars->drain);
     wait_drain(&bars->drain, 0);
+    pa.flush(true);
 }
 
 // ------------------------------------------------------------------ group scratch
@@ -266,20 +343,12 @@ struct WgScratch {          // one per epilogue warpgroup
     uint32_t hist[kNbCompact];
 };
 
-struct FinScratch {         // the finalizer's
-    GroupSmall gs;
-    int gather_n;
-    int pad[3];
-    uint32_t hist[kNbFinal];
-    uint64_t gather[kGatherMax];
-    uint64_t stage[kMaxTopk];
-};
-
 // ------------------------------------------------------------------ compaction
 // Cuts a query's list back when it could overflow: keeps every key whose
-// bucket is at or above the bucket of the k-th largest key (a superset of the
-// top k), or -- when the score range is degenerate or that bucket is too full
-// -- the radix-exact top k plus slack.  Updates cnt, bound and min_ord.
+// bucket (over the list's own [min, max] score range) is at or above the
+// bucket of the k-th largest key -- a superset of the top k -- or, when the
+// range is degenerate or that bucket is too full, the radix-exact top k plus
+// slack.  Updates cnt and raises bound to the smallest kept score.
 __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, WgScratch *sc,
                              int bar, int tid)
 {
@@ -290,7 +359,9 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
         const int j = i * kGroupThreads + tid;
         e[i] = j < n ? list[j] : 0ull;
     }
-    const BucketMap bm = bucket_map(st.min_ord, st.max_ord, kNbCompact);
+    uint32_t mn_all, mx_all;
+    group_ord_range<kGroupThreads, kEpt>(e, &sc->gs, bar, tid, &mn_all, &mx_all);
+    const BucketMap bm = bucket_map_unit(mn_all, mx_all);
     bool done = false;
     uint32_t newmin = 0xFFFFFFFFu;
     int kept = 0;
@@ -301,7 +372,7 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
 #pragma unroll
         for (int i = 0; i < kEpt; ++i)
             if (e[i] != 0)
-                atomicAdd(&sc->hist[bucket_of(key_score(e[i]), bm, kNbCompact)], 1u);
+                atomicAdd(&sc->hist[bucket_of_sqrt(key_score(e[i]), bm, kNbCompact)], 1u);
         named_bar_sync(bar, kGroupThreads);
         bucket_boundary<kGroupThreads, kNbCompact>(sc->hist, p.topk, false, &sc->gs, bar, tid);
         const int bstar = sc->gs.bcast[0];
@@ -310,18 +381,19 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
         if (cand_kept <= p.cap - 2 * kTileKeys) {
             int mine = 0;
             uint32_t mn = 0xFFFFFFFFu;
-            bool keep[kEpt];
+            uint32_t keep = 0;
 #pragma unroll
             for (int i = 0; i < kEpt; ++i) {
-                keep[i] = e[i] != 0 && bucket_of(key_score(e[i]), bm, kNbCompact) >= bstar;
-                mine += keep[i] ? 1 : 0;
-                mn = keep[i] ? min(mn, key_ord(e[i])) : mn;
+                const bool k = e[i] != 0 && bucket_of_sqrt(key_score(e[i]), bm, kNbCompact) >= bstar;
+                keep |= k ? (1u << i) : 0u;
+                mine += k ? 1 : 0;
+                mn = k ? min(mn, key_ord(e[i])) : mn;
             }
             int total;
             int off = group_excl_scan<kGroupThreads>(mine, &sc->gs, bar, tid, &total);
 #pragma unroll
             for (int i = 0; i < kEpt; ++i)
-                if (keep[i])
+                if (keep & (1u << i))
                     list[off++] = e[i];
             newmin = group_min_u32<kGroupThreads>(mn, &sc->gs, bar, tid);
             kept = total;
@@ -338,13 +410,169 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
     if (tid == 0) {
         st.cnt = kept;
         st.bound = max(st.bound, newmin);
-        st.min_ord = newmin;
     }
     named_bar_sync(bar, kGroupThreads);
 }
 
+// ------------------------------------------------------------------ emission
+// Appends this warp's surviving (score, key) pairs of Q queries to their
+// candidate lists: one ballot per query, the lane-0 atomics back to back.
+// Query j's list starts at lbase + j * lstride.
+template <int Q>
+__device__ __forceinline__ void emit_batch(const float *sc, int j0, int s, float kscale,
+                                           QueryState *qs, uint64_t *lbase, size_t lstride,
+                                           int lane)
+{
+    uint32_t ord[Q];
+    unsigned bal[Q];
+    int base[Q];
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+        const QueryState st = qs[j0 + q];
+        ord[q] = ord_of_score(sc[q] * kscale);
+        bal[q] = __ballot_sync(0xffffffffu, s < st.vis_end && ord[q] >= st.bound);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < Q; ++q)
+            base[q] = bal[q] ? atomicAdd(&qs[j0 + q].cnt, __popc(bal[q])) : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+        base[q] = __shfl_sync(0xffffffffu, base[q], 0);
+        if (bal[q] & (1u << lane))
+            lbase[static_cast<size_t>(j0 + q) * lstride + base[q] +
+                  __popc(bal[q] & lanemask_lt())] = make_key(ord[q], static_cast<uint32_t>(s));
+    }
+}
+
+// ------------------------------------------------------------------ fast tile math
+template <int FC> struct Ld16x256;
+template <> struct Ld16x256<64> {
+    static __device__ __forceinline__ void ld(uint32_t a, uint32_t (&v)[32]) { tmem_ld_16x256b_x8(a, v); }
+};
+template <> struct Ld16x256<128> {
+    static __device__ __forceinline__ void ld(uint32_t a, uint32_t (&v)[64]) { tmem_ld_16x256b_x16(a, v); }
+};
+
+// This thread's head weights for a warpgroup that reads FC columns holding FQ
+// queries: weight 2i+e belongs to column 8i + 2(lane%4) + e.
+template <int FC, int FQ>
+__device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int j0, int lane,
+                                            float (&wr)[FC / 4])
+{
+    constexpr int RPQ = FC / 8 / FQ;  // 8-column repetitions per query
+#pragma unroll
+    for (int i = 0; i < FC / 8; ++i) {
+        const int j = j0 + i / RPQ;
+        const int h = 8 * (i % RPQ) + 2 * (lane & 3);
+        float a = 0.0f, b = 0.0f;
+        if (j < it.nq) {
+            const float *src = p.w + (static_cast<size_t>(it.b) * p.S + it.q0 + j) * p.H + h;
+            a = src[0];
+            b = src[1];
+        }
+        wr[2 * i] = a;
+        wr[2 * i + 1] = b;
+    }
+}
+
+// Scores of FQ queries for one key per thread.  The warp's two 16-lane loads
+// cover its 32 keys; thread t holds columns 8i + 2(t%4) + {0,1} of keys
+// t/4 + {0, 8, 16, 24}.  After the loads land the accumulator slot is released
+// (one arrive per warp).  Each thread then forms per-key partial sums over its
+// columns; the quad (threads sharing t/4) exchanges halves twice so that
+// thread t ends with the complete scores of key row 16*((t>>1)&1) + 8*(t&1)
+// + t/4 of the warp's 32.
+template <int FC, int FQ>
+__device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float (&wr)[FC / 4],
+                                                 uint64_t *acc_empty, int lane, float (&F)[FQ])
+{
+    constexpr int NV = FC / 2;
+    constexpr int REPS = FC / 8;
+    constexpr int RPQ = REPS / FQ;
+    uint32_t va[NV], vb[NV];
+    __syncwarp();
+    Ld16x256<FC>::ld(taddr, va);
+    Ld16x256<FC>::ld(taddr + (16u << 16), vb);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        reg_fence(va[i]);
+        reg_fence(vb[i]);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(acc_empty);
+    float P[4][FQ][2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int j = 0; j < FQ; ++j)
+            P[k][j][0] = P[k][j][1] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < REPS; ++i) {
+        const int j = i / RPQ;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float w = wr[2 * i + e];
+                P[sub][j][e] =
+                    fmaf(fmaxf(__uint_as_float(va[4 * i + 2 * sub + e]), 0.0f), w, P[sub][j][e]);
+                P[2 + sub][j][e] = fmaf(fmaxf(__uint_as_float(vb[4 * i + 2 * sub + e]), 0.0f), w,
+                                        P[2 + sub][j][e]);
+            }
+        }
+    }
+    const bool b1 = (lane >> 1) & 1;
+    const bool b0 = lane & 1;
+#pragma unroll
+    for (int j = 0; j < FQ; ++j) {
+        float R[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const float lo = P[m][j][0] + P[m][j][1];          // key m (first 16 lanes)
+            const float hi = P[2 + m][j][0] + P[2 + m][j][1];  // key 2+m (last 16 lanes)
+            const float send = b1 ? lo : hi;
+            const float keep = b1 ? hi : lo;
+            R[m] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        }
+        const float send = b0 ? R[0] : R[1];
+        const float keep = b0 ? R[1] : R[0];
+        F[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+}
+
+// ------------------------------------------------------------------ generic tile math
+// One 32-column TMEM chunk: sum over the chunk's heads of w * ReLU(logit),
+// four independent accumulators.
+__device__ __forceinline__ float chunk_dot(const uint32_t (&v)[32], const float *wc)
+{
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        const float4 w4 = *reinterpret_cast<const float4 *>(wc + i);
+        a0 = fmaf(fmaxf(__uint_as_float(v[i + 0]), 0.0f), w4.x, a0);
+        a1 = fmaf(fmaxf(__uint_as_float(v[i + 1]), 0.0f), w4.y, a1);
+        a2 = fmaf(fmaxf(__uint_as_float(v[i + 2]), 0.0f), w4.z, a2);
+        a3 = fmaf(fmaxf(__uint_as_float(v[i + 3]), 0.0f), w4.w, a3);
+    }
+    return (a0 + a1) + (a2 + a3);
+}
+
+__device__ __forceinline__ void fence_regs(uint32_t (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        reg_fence(v[i]);
+}
+
 // ------------------------------------------------------------------ epilogue
-template <bool kHeadsGe32>
+// FC > 0: fast path for FC columns and FQ queries per warpgroup.  FC == 0:
+// generic path (kHeadsGe32 tells whether a query spans whole 32-column chunks).
+template <int FC, int FQ, bool kHeadsGe32>
 __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uint32_t tmem_base,
                              const WaitCtl &ctl, int wg)
 {
@@ -353,20 +581,32 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
     const int lane = threadIdx.x & 31;
     const int bar = wg == 0 ? kBarWg0 : kBarWg1;
     const int quarter = warp & 3;             // TMEM lanes this warp may read
-    const int key_local = quarter * 32 + lane;
     float *w_s = reinterpret_cast<float *>(smem + p.off_w);
-    QueryState *qs_all = reinterpret_cast<QueryState *>(smem + p.off_state);
+    QueryState *qs = reinterpret_cast<QueryState *>(smem + p.off_state);
     WgScratch *sc = reinterpret_cast<WgScratch *>(smem + p.off_wg + wg * p.wg_bytes);
-    uint64_t *cand_cta = p.cand + static_cast<size_t>(blockIdx.x) * 2 * p.qps * p.cap;
     const uint32_t bound0 = p.mode == 1 ? 0x80000001u : 0u; // gate: score > 0
     const int j0 = wg * p.qpw;                 // first query slot this group owns
     const int col0 = j0 * p.H;                 // first TMEM column it reads
     const int ncols = p.qpw * p.H;             // TMEM columns it reads
-    const int nchunk = ncols / 32;             // in 32-column chunks
-    int acc_use = 0, it_count = 0;
-    constexpr int kWRegs = kSlotCols / kGroupThreads;
+    const int nchunk = ncols / 32;             // in 32-column chunks (generic path)
+    const int cpq_shift = p.H >= 32 ? __ffs(p.H / 32) - 1 : 0;
+    const int h_shift = __ffs(p.H) - 1;
+    const size_t lstride = static_cast<size_t>(p.nsplit) * p.cap;
+    // the key row (of the warp's 32) whose scores this thread ends up with
+    const int key_local =
+        FC > 0 ? quarter * 32 + 16 * ((lane >> 1) & 1) + 8 * (lane & 1) + (lane >> 2)
+               : quarter * 32 + lane;
+    int acc_use = 0;
+    ProfAcc pa;
+    Prof pf, pt;
+    const bool rec = wg == 0 && tid == 0;
+    pt.start();
+
+    // Generic path: the group's weights go through shared memory, loaded into
+    // registers one item ahead.
+    constexpr int kWRegs = FC > 0 ? 1 : kSlotCols / kGroupThreads;
     float wnext[kWRegs];
-    {
+    if (FC == 0) {
         const Item it0 = decode_item(p, blockIdx.x);
         const size_t row = static_cast<size_t>(it0.b) * p.S + it0.q0;
         for (int r = 0; r < kWRegs; ++r) {
@@ -376,40 +616,29 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                            : 0.0f;
         }
     }
+    float wr[FC > 0 ? FC / 4 : 1];
 
+    bool ok = true;
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
-        const int buf = it_count & 1;
-        QueryState *qs = qs_all + buf * p.qps;
-        uint64_t *lists = cand_cta + static_cast<size_t>(buf) * p.qps * p.cap;
-        // The finalizer must be done with this list buffer (item it_count - 2).
-        bool ok = wait_bounded(&bars->fin_empty[buf], ((it_count >> 1) & 1) ^ 1, ctl,
-                               kRoleEpilogue, id);
-        ok = group_all(bar, kGroupThreads, ok);
-        if (!ok) {
-            *ctl.abort = 1;
-            break;
-        }
+        uint64_t *lbase = p.lists + (static_cast<size_t>(it.lrow) * p.nsplit + it.split) * p.cap;
         for (int j = j0 + tid; j < j0 + p.qpw; j += kGroupThreads) {
             const int i = it.q0 + j;
             QueryState st;
             st.cnt = 0;
             st.bound = bound0;
-            st.min_ord = 0xFFFFFFFFu;
-            st.max_ord = 0u;
             st.vis_end = i < p.S ? visible_count(p, static_cast<long long>(i) + p.q_offset) : 0;
-            st.pad[0] = st.pad[1] = st.pad[2] = 0;
+            st.pad = 0;
             qs[j] = st;
         }
-        // This group's head weights for the item: registers loaded one item
-        // ahead, stored to the group's own columns of w_s (nothing else reads
-        // them), then the next item's loads are issued.
-        for (int r = 0; r < kWRegs; ++r) {
-            const int c = tid + r * kGroupThreads;
-            if (c < ncols)
-                w_s[col0 + c] = wnext[r];
-        }
-        {
+        if constexpr (FC > 0) {
+            fast_load_w<FC, FQ>(p, it, j0, lane, wr);
+        } else {
+            for (int r = 0; r < kWRegs; ++r) {
+                const int c = tid + r * kGroupThreads;
+                if (c < ncols)
+                    w_s[col0 + c] = wnext[r];
+            }
             const int nid = id + gridDim.x;
             if (nid < p.n_items) {
                 const Item nx = decode_item(p, nid);
@@ -428,265 +657,105 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
             if (p.key_fp8 && s < p.T)
                 kscale = p.k_scale[static_cast<size_t>(it.b) * p.T + s];
             const int slot = acc_use & 1;
+            pf.start();
             ok = wait_bounded(&bars->acc_full[slot], (acc_use >> 1) & 1, ctl, kRoleEpilogue, id);
-            ok = group_all(bar, kGroupThreads, ok);
-            if (!ok)
-                break;
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   slot * kSlotCols + col0;
-            const float *wsub = w_s + col0;
-
-            auto emit = [&](int jq, float score) {
-                QueryState &st = qs[jq];
-                const uint32_t ord = ord_of_score(score * kscale);
-                const bool pass = s < st.vis_end && ord >= st.bound;
-                const unsigned bal = __ballot_sync(0xffffffffu, pass);
-                if (bal) {
-                    const uint32_t mx = __reduce_max_sync(0xffffffffu, pass ? ord : 0u);
-                    const uint32_t mn = __reduce_min_sync(0xffffffffu, pass ? ord : 0xFFFFFFFFu);
-                    int base = 0;
-                    if (lane == 0) {
-                        base = atomicAdd(&st.cnt, __popc(bal));
-                        atomicMax(&st.max_ord, mx);
-                        atomicMin(&st.min_ord, mn);
-                    }
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    if (pass)
-                        lists[static_cast<size_t>(jq) * p.cap + base + __popc(bal & lanemask_lt())] =
-                            make_key(ord, static_cast<uint32_t>(s));
-                }
-            };
-
-            float acc = 0.0f;
-            uint32_t v[32];
-            __syncwarp();
-            tmem_ld_32x32b_x32(taddr, v);
-            for (int c = 0; c < nchunk; ++c) {
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    reg_fence(v[i]);
-                float x[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    x[i] = fmaxf(__uint_as_float(v[i]), 0.0f);
-                if (c + 1 < nchunk) {
-                    __syncwarp();
-                    tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
-                }
-                const float *wc = wsub + c * 32;
-                if (kHeadsGe32) {
-                    // packed fp32 FMA over pairs of heads
-                    unsigned long long a0 = 0ull, a1 = 0ull;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 w4 = *reinterpret_cast<const float4 *>(wc + i);
-                        unsigned long long xa, xb, wa, wb;
-                        asm("mov.b64 %0, {%1, %2};" : "=l"(xa) : "f"(x[i]), "f"(x[i + 1]));
-                        asm("mov.b64 %0, {%1, %2};" : "=l"(xb) : "f"(x[i + 2]), "f"(x[i + 3]));
-                        asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(w4.x), "f"(w4.y));
-                        asm("mov.b64 %0, {%1, %2};" : "=l"(wb) : "f"(w4.z), "f"(w4.w));
-                        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a0) : "l"(xa), "l"(wa));
-                        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a1) : "l"(xb), "l"(wb));
-                    }
-                    float p0, p1, p2, p3;
-                    asm("mov.b64 {%0, %1}, %2;" : "=f"(p0), "=f"(p1) : "l"(a0));
-                    asm("mov.b64 {%0, %1}, %2;" : "=f"(p2), "=f"(p3) : "l"(a1));
-                    acc += (p0 + p1) + (p2 + p3);
-                    if (((c + 1) * 32) % p.H == 0) {
-                        emit(j0 + (c * 32) / p.H, acc);
-                        acc = 0.0f;
-                    }
+            // the TMEM loads below are warp-collective: agree on the outcome first
+            ok = __all_sync(0xffffffffu, ok);
+            pf.add(pa, kPfEpiAccFull, rec);
+            pf.count(pa, kPfEpiTiles, rec);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                       slot * kSlotCols + col0;
+                pf.start();
+                if constexpr (FC > 0) {
+                    float F[FQ];
+                    fast_tile_scores<FC, FQ>(taddr, wr, &bars->acc_empty[slot], lane, F);
+                    emit_batch<FQ>(F, j0, s, kscale, qs, lbase, lstride, lane);
                 } else {
-                    // H < 32 (a power of two): each 32-column chunk holds 32/H queries
+                    // One chunk at a time, each query emitted as it completes.
+                    auto emit = [&](int jq, float score) {
+                        QueryState &st = qs[jq];
+                        const uint32_t ord = ord_of_score(score * kscale);
+                        const bool pass = s < st.vis_end && ord >= st.bound;
+                        const unsigned bal = __ballot_sync(0xffffffffu, pass);
+                        if (bal) {
+                            int base = 0;
+                            if (lane == 0)
+                                base = atomicAdd(&st.cnt, __popc(bal));
+                            base = __shfl_sync(0xffffffffu, base, 0);
+                            if (pass)
+                                lbase[static_cast<size_t>(jq) * lstride + base +
+                                      __popc(bal & lanemask_lt())] =
+                                    make_key(ord, static_cast<uint32_t>(s));
+                        }
+                    };
+                    const float *wsub = w_s + col0;
+                    float acc = 0.0f;
+                    uint32_t v[32];
+                    for (int c = 0; c < nchunk; ++c) {
+                        __syncwarp();
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        tmem_ld_wait();
+                        fence_regs(v);
+                        const float *wc = wsub + c * 32;
+                        if (kHeadsGe32) {
+                            acc += chunk_dot(v, wc);
+                            if (((c + 1) & ((1 << cpq_shift) - 1)) == 0) {
+                                emit(j0 + (c >> cpq_shift), acc);
+                                acc = 0.0f;
+                            }
+                        } else {
+                            // H < 32 (a power of two): each 32-column chunk holds 32/H queries
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        acc = fmaf(x[i], wc[i], acc);
-                        if (((i + 1) & (p.H - 1)) == 0) {
-                            emit(j0 + (c * 32 + i) / p.H, acc);
-                            acc = 0.0f;
+                            for (int i = 0; i < 32; ++i) {
+                                acc = fmaf(fmaxf(__uint_as_float(v[i]), 0.0f), wc[i], acc);
+                                if (((i + 1) & (p.H - 1)) == 0) {
+                                    emit(j0 + ((c * 32 + i) >> h_shift), acc);
+                                    acc = 0.0f;
+                                }
+                            }
                         }
                     }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->acc_empty[slot]);
                 }
+                pf.add(pa, kPfEpiMath, rec);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars->acc_empty[slot]);
             ++acc_use;
-            named_bar_sync(bar, kGroupThreads);
+            pf.start();
+            ok = group_all(bar, kGroupThreads, ok);
+            pf.add(pa, kPfEpiTileBar, rec);
+            if (!ok)
+                break;
             // Cut back any list that the next tile could overflow.
             for (int jq = j0; jq < j0 + p.qpw; ++jq) {
-                if (qs[jq].cnt > p.cap - kTileKeys)
-                    compact_list(p, lists + static_cast<size_t>(jq) * p.cap, qs[jq], sc, bar, tid);
+                if (qs[jq].cnt > p.cap - kTileKeys) {
+                    pf.start();
+                    compact_list(p, lbase + static_cast<size_t>(jq) * lstride, qs[jq], sc, bar, tid);
+                    pf.add(pa, kPfEpiCompact, rec);
+                    pf.count(pa, kPfEpiCompactCount, rec);
+                }
             }
         }
         if (!ok) {
             *ctl.abort = 1;
             break;
         }
-        // Hand the finished lists to the finalizer.
-        mbar_arrive(&bars->fin_full[buf]);
-        ++it_count;
-    }
-}
-
-// ------------------------------------------------------------------ finalizer
-// Exact top-k of one finished list, sorted by (score desc, index asc):
-// histogram over [min, max] score buckets, resolve the boundary bucket in
-// place, counting-sort the selected keys by bucket and sort each (small)
-// bucket.  Degenerate cases take the radix-exact path and a bitonic sort.
-// Returns the number of keys, in order, in sc->stage.
-__device__ int final_select(const Params &p, const uint64_t *list, const QueryState &st,
-                            FinScratch *sc, int bar, int tid)
-{
-    const int n = st.cnt;
-    const int K = p.topk;
-    const int kept = min(n, K);
-    if (kept == 0)
-        return 0;
-    uint64_t e[kEpt];
-#pragma unroll
-    for (int i = 0; i < kEpt; ++i) {
-        const int j = i * kGroupThreads + tid;
-        e[i] = j < n ? list[j] : 0ull;
-    }
-    const BucketMap bm = bucket_map(st.min_ord, st.max_ord, kNbFinal);
-    if (bm.ok) {
-        for (int i = tid; i < kNbFinal; i += kGroupThreads)
-            sc->hist[i] = 0;
-        if (tid == 0)
-            sc->gather_n = 0;
+        // Publish the list lengths (rows past the end of the batch get 0).
+        for (int j = j0 + tid; j < j0 + p.qpw; j += kGroupThreads)
+            p.counts[static_cast<size_t>(it.lrow + j) * p.nsplit + it.split] =
+                j < it.nq ? qs[j].cnt : 0;
         named_bar_sync(bar, kGroupThreads);
-#pragma unroll
-        for (int i = 0; i < kEpt; ++i)
-            if (e[i] != 0)
-                atomicAdd(&sc->hist[bucket_of(key_score(e[i]), bm, kNbFinal)], 1u);
-        named_bar_sync(bar, kGroupThreads);
-        bucket_boundary<kGroupThreads, kNbFinal>(sc->hist, kept, true, &sc->gs, bar, tid);
-        const int bstar = sc->gs.bcast[0];
-        const int above = sc->gs.bcast[1];
-        const int inb = sc->gs.bcast[2];
-        const int biggest = sc->gs.bcast[3];
-        named_bar_sync(bar, kGroupThreads);
-        if (biggest <= kBucketSortMax && inb <= kGatherMax) {
-            const int r = kept - above; // keys taken from the boundary bucket
-            // gather the boundary bucket when only part of it is taken
-            if (r < inb) {
-#pragma unroll
-                for (int i = 0; i < kEpt; ++i)
-                    if (e[i] != 0 && bucket_of(key_score(e[i]), bm, kNbFinal) == bstar)
-                        sc->gather[atomicAdd(&sc->gather_n, 1)] = e[i];
-                named_bar_sync(bar, kGroupThreads);
-            }
-            // counting-sort scatter: hist[b] holds the next free slot of bucket b
-#pragma unroll
-            for (int i = 0; i < kEpt; ++i) {
-                if (e[i] == 0)
-                    continue;
-                const int b = bucket_of(key_score(e[i]), bm, kNbFinal);
-                bool sel = b > bstar;
-                if (b == bstar) {
-                    if (r < inb) {
-                        int rank = 0;
-                        for (int g = 0; g < inb; ++g)
-                            rank += sc->gather[g] > e[i] ? 1 : 0;
-                        sel = rank < r;
-                    } else {
-                        sel = true;
-                    }
-                }
-                if (sel)
-                    sc->stage[atomicAdd(&sc->hist[b], 1u)] = e[i];
-            }
-            named_bar_sync(bar, kGroupThreads);
-            // per-bucket insertion sort, descending: bucket b spans
-            // [end of bucket b+1, end of bucket b) after the scatter
-            for (int b = tid; b < kNbFinal; b += kGroupThreads) {
-                if (b < bstar)
-                    continue;
-                const int end = static_cast<int>(sc->hist[b]);
-                const int beg = b + 1 < kNbFinal ? static_cast<int>(sc->hist[b + 1]) : 0;
-                for (int x = beg + 1; x < end; ++x) {
-                    const uint64_t key = sc->stage[x];
-                    int y = x - 1;
-                    while (y >= beg && sc->stage[y] < key) {
-                        sc->stage[y + 1] = sc->stage[y];
-                        --y;
-                    }
-                    sc->stage[y + 1] = key;
-                }
-            }
-            named_bar_sync(bar, kGroupThreads);
-            return kept;
-        }
     }
-    // exact fallback: radix select + bitonic sort
-    const int P = pow2_at_least(kept);
-    uint64_t L = 1;
-    if (n > K) {
-        int k2;
-        L = radix_bound<kGroupThreads, kEpt>(e, K, 0, sc->hist, &sc->gs, bar, tid, &k2);
-    }
-    uint32_t mn;
-    const int total = write_kept<kGroupThreads, kEpt>(e, L, sc->stage, &sc->gs, bar, tid, &mn);
-    for (int i = total + tid; i < P; i += kGroupThreads)
-        sc->stage[i] = 0ull;
-    named_bar_sync(bar, kGroupThreads);
-    bitonic_sort_desc<kGroupThreads>(sc->stage, P, bar, tid);
-    return kept;
-}
-
-__device__ void run_finalizer(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl)
-{
-    const int tid = threadIdx.x - 320; // warps 10..13
-    QueryState *qs_all = reinterpret_cast<QueryState *>(smem + p.off_state);
-    FinScratch *sc = reinterpret_cast<FinScratch *>(smem + p.off_fin);
-    const uint64_t *cand_cta = p.cand + static_cast<size_t>(blockIdx.x) * 2 * p.qps * p.cap;
-    int it_count = 0;
-    for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
-        const Item it = decode_item(p, id);
-        const int buf = it_count & 1;
-        bool ok = wait_bounded(&bars->fin_full[buf], (it_count >> 1) & 1, ctl, kRoleFinal, id);
-        ok = group_all(kBarFin, kGroupThreads, ok);
-        if (!ok) {
-            *ctl.abort = 1;
-            break;
-        }
-        const QueryState *qs = qs_all + buf * p.qps;
-        const uint64_t *lists = cand_cta + static_cast<size_t>(buf) * p.qps * p.cap;
-        for (int j = 0; j < it.nq; ++j) {
-            const QueryState st = qs[j];
-            const int kept = final_select(p, lists + static_cast<size_t>(j) * p.cap, st, sc,
-                                          kBarFin, tid);
-            const size_t row = static_cast<size_t>(it.b) * p.S + it.q0 + j;
-            if (p.nsplit == 1) {
-                for (int slot = tid; slot < p.topk; slot += kGroupThreads) {
-                    const size_t o = row * p.topk + slot;
-                    if (slot < kept) {
-                        const uint64_t key = sc->stage[slot];
-                        p.out_idx[o] = key_index(key);
-                        p.out_score[o] = key_score(key);
-                    } else {
-                        p.out_idx[o] = -1;
-                        p.out_score[o] = -__int_as_float(0x7f800000);
-                    }
-                }
-            } else {
-                uint64_t *dst = p.part + (row * p.nsplit + it.split) * p.topk;
-                for (int slot = tid; slot < p.topk; slot += kGroupThreads)
-                    dst[slot] = slot < kept ? sc->stage[slot] : 0ull;
-            }
-            named_bar_sync(kBarFin, kGroupThreads);
-        }
-        mbar_arrive(&bars->fin_empty[buf]);
-        ++it_count;
-    }
+    pt.add(pa, kPfEpiTotal, rec);
+    pa.flush(rec);
 }
 
 // ------------------------------------------------------------------ kernel
-template <bool kHeadsGe32>
+template <int FC, int FQ, bool kHeadsGe32>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_topk_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK, const Params p)
@@ -710,8 +779,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->acc_full[s], 1);
             mbar_init(&bars->acc_empty[s], epi_warps);
-            mbar_init(&bars->fin_full[s], 32 * epi_warps);
-            mbar_init(&bars->fin_empty[s], kGroupThreads);
         }
         bars->abort = 0;
         fence_mbar_init();
@@ -735,12 +802,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0)
             run_mma(p, smem, bars, tmem_base, ctl);
     } else if (warp < 6) {
-        run_epilogue<kHeadsGe32>(p, smem, bars, tmem_base, ctl, 0);
-    } else if (warp < 10) {
-        if (p.n_wg == 2)
-            run_epilogue<kHeadsGe32>(p, smem, bars, tmem_base, ctl, 1);
+        run_epilogue<FC, FQ, kHeadsGe32>(p, smem, bars, tmem_base, ctl, 0);
     } else {
-        run_finalizer(p, smem, bars, ctl);
+        if (p.n_wg == 2)
+            run_epilogue<FC, FQ, kHeadsGe32>(p, smem, bars, tmem_base, ctl, 1);
     }
 
     tc_fence_before();
@@ -749,62 +814,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         __syncwarp();
         tmem_dealloc(tmem_base, 2 * kSlotCols);
-    }
-}
-
-// ------------------------------------------------------------------ split merge
-// Merges the nsplit partial lists of one query row into its final top-k:
-// "StreamIndex ...", abstract (a partition-merge top-k that never materialises
-// the full score tensor); here the partitions are key ranges of one query.
-constexpr int kMergeThreads = 256;
-constexpr int kMergeEpt = 32; // nsplit * topk <= 8192
-
-__global__ void __launch_bounds__(kMergeThreads)
-    merge_splits_kernel(const uint64_t *__restrict__ part, int rows, int nsplit, int topk,
-                        int32_t *__restrict__ out_idx, float *__restrict__ out_score)
-{
-    __shared__ GroupSmall gs;
-    __shared__ uint32_t hist[256];
-    __shared__ uint64_t sortbuf[kMaxTopk];
-    const int tid = threadIdx.x;
-    for (int row = blockIdx.x; row < rows; row += gridDim.x) {
-        const uint64_t *src = part + static_cast<size_t>(row) * nsplit * topk;
-        const int n_all = nsplit * topk;
-        uint64_t e[kMergeEpt];
-        int mine = 0;
-#pragma unroll
-        for (int i = 0; i < kMergeEpt; ++i) {
-            const int x = i * kMergeThreads + tid;
-            e[i] = x < n_all ? src[x] : 0ull;
-            mine += e[i] != 0;
-        }
-        int n;
-        group_excl_scan<kMergeThreads>(mine, &gs, 0, tid, &n);
-        const int kept = min(n, topk);
-        const int P = pow2_at_least(kept);
-        uint64_t L = 1;
-        if (n > topk) {
-            int k2;
-            L = radix_bound<kMergeThreads, kMergeEpt>(e, topk, 0, hist, &gs, 0, tid, &k2);
-        }
-        uint32_t mn;
-        const int total = write_kept<kMergeThreads, kMergeEpt>(e, L, sortbuf, &gs, 0, tid, &mn);
-        for (int i = total + tid; i < P; i += kMergeThreads)
-            sortbuf[i] = 0ull;
-        __syncthreads();
-        bitonic_sort_desc<kMergeThreads>(sortbuf, P, 0, tid);
-        for (int slot = tid; slot < topk; slot += kMergeThreads) {
-            const size_t o = static_cast<size_t>(row) * topk + slot;
-            if (slot < kept) {
-                const uint64_t key = sortbuf[slot];
-                out_idx[o] = key_index(key);
-                out_score[o] = key_score(key);
-            } else {
-                out_idx[o] = -1;
-                out_score[o] = -__int_as_float(0x7f800000);
-            }
-        }
-        __syncthreads();
     }
 }
 

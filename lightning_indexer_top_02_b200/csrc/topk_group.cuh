@@ -117,6 +117,58 @@ __device__ __forceinline__ uint32_t group_min_u32(uint32_t v, GroupSmall *gs, in
     return r;
 }
 
+// Smallest and largest score order image among the group's non-zero keys.
+template <int NT, int EPT>
+__device__ __forceinline__ void group_ord_range(const uint64_t (&e)[EPT], GroupSmall *gs, int bar,
+                                                int tid, uint32_t *mn, uint32_t *mx)
+{
+    const int lane = tid & 31, wid = tid >> 5;
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+        if (e[i] != 0) {
+            lo = min(lo, key_ord(e[i]));
+            hi = max(hi, key_ord(e[i]));
+        }
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+        gs->warp_sums[wid] = lo;
+        gs->warp_sums[16 + wid] = hi;
+    }
+    named_bar_sync(bar, NT);
+    uint32_t a = 0xFFFFFFFFu, b = 0u;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        a = min(a, gs->warp_sums[w]);
+        b = max(b, gs->warp_sums[16 + w]);
+    }
+    named_bar_sync(bar, NT);
+    *mn = a;
+    *mx = b;
+}
+
+// Warp-aggregated counter increment: lanes with the same idx share one
+// atomic.  Returns, for active lanes, the counter's old value plus the lane's
+// rank among its peers (a unique slot).  All 32 lanes must call it.
+__device__ __forceinline__ uint32_t agg_atomic_add(uint32_t *counters, int idx, bool active)
+{
+    const unsigned act = __ballot_sync(0xffffffffu, active);
+    uint32_t res = 0;
+    if (active) {
+        const int lane = threadIdx.x & 31;
+        const unsigned peers = __match_any_sync(act, idx);
+        const int leader = __ffs(peers) - 1;
+        uint32_t base = 0;
+        if (lane == leader)
+            base = atomicAdd(&counters[idx], static_cast<uint32_t>(__popc(peers)));
+        base = __shfl_sync(peers, base, leader);
+        res = base + static_cast<uint32_t>(__popc(peers & lanemask_lt()));
+    }
+    return res;
+}
+
 // ---------------------------------------------------------------------------- radix (exact)
 
 // Radix select over the group's keys (EPT per thread, 0 = empty), most
@@ -349,6 +401,94 @@ __device__ void bucket_boundary(uint32_t *hist, int need, bool write_above, Grou
         gs->bcast[3] = static_cast<int>(m);
     }
     named_bar_sync(bar, NT);
+}
+
+// Square-root bucket map: b(x) = floor(NB * sqrt((x - lo) / (hi - lo))).
+// Still monotone (each step is), but it spreads the dense low end of a
+// candidate list -- scores just above the admission bound -- over many more
+// buckets than a linear map, so fewer keys share a bucket (and an atomic).
+__device__ __forceinline__ int bucket_of_sqrt(float s, const BucketMap &m, int NB)
+{
+    const float u = (s - m.lo) * m.inv; // m.inv = 1 / span for this map
+    const float r = sqrtf(u > 0.0f ? u : 0.0f) * static_cast<float>(NB);
+    int b = static_cast<int>(r);
+    return b > NB - 1 ? NB - 1 : b;
+}
+
+__device__ __forceinline__ BucketMap bucket_map_unit(uint32_t min_ord, uint32_t max_ord)
+{
+    BucketMap m;
+    const float lo = score_of_ord(min_ord);
+    const float hi = score_of_ord(max_ord);
+    const float span = hi - lo;
+    m.lo = lo;
+    m.inv = 1.0f / span;
+    m.ok = max_ord > min_ord && span > 0.0f && isfinite(span) && isfinite(m.inv) && isfinite(lo);
+    return m;
+}
+
+// ---------------------------------------------------------------------------- bitonic in registers
+// 64-bit compare-exchange keeping the larger key in a when `big_first`.
+__device__ __forceinline__ void cex(uint64_t &a, uint64_t &b, bool big_first)
+{
+    const bool sw = big_first ? (a < b) : (a > b);
+    const uint64_t x = sw ? b : a;
+    const uint64_t y = sw ? a : b;
+    a = x;
+    b = y;
+}
+
+// Sorts P = 128 * EPT keys held by a 128-thread group (element j = tid * EPT
+// + r lives in a[r] of thread tid) into descending order.  Pairs closer than
+// EPT are exchanged inside a thread, pairs within a warp through shuffles,
+// and the few cross-warp steps through `buf` (P keys of shared memory).
+template <int EPT>
+__device__ void bitonic_sort_regs(uint64_t (&a)[EPT], uint64_t *buf, int bar, int tid)
+{
+    constexpr int P = 128 * EPT;
+    const int lane = tid & 31;
+    const int base = tid * EPT;
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int s = k >> 1; s >= EPT; s >>= 1) {
+            // partner lives in another thread: lane ^ (s / EPT), or another warp
+            const bool lower = (base & s) == 0;
+            const bool desc = (base & k) == 0;
+            const bool keep_big = lower == desc;
+            if (s < 32 * EPT) {
+                const int m = s / EPT;
+#pragma unroll
+                for (int r = 0; r < EPT; ++r) {
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, a[r], m);
+                    a[r] = keep_big ? (a[r] > o ? a[r] : o) : (a[r] < o ? a[r] : o);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < EPT; ++r)
+                    buf[base + r] = a[r];
+                named_bar_sync(bar, 128);
+#pragma unroll
+                for (int r = 0; r < EPT; ++r) {
+                    const uint64_t o = buf[(base + r) ^ s];
+                    a[r] = keep_big ? (a[r] > o ? a[r] : o) : (a[r] < o ? a[r] : o);
+                }
+                named_bar_sync(bar, 128);
+            }
+            (void)lane;
+        }
+        // partner in the same thread
+#pragma unroll
+        for (int sc = EPT / 2; sc >= 1; sc >>= 1) {
+            if (sc < k) {
+#pragma unroll
+                for (int r = 0; r < EPT; ++r) {
+                    if ((r & sc) == 0) {
+                        const bool desc = ((base + r) & k) == 0;
+                        cex(a[r], a[r | sc], desc);
+                    }
+                }
+            }
+        }
+    }
 }
 
 __host__ __device__ constexpr int pow2_at_least(int x)

@@ -82,10 +82,11 @@ def test_split_shape_and_gate(lib):
 
 
 def test_too_large_is_refused(lib):
-    """The batched-decode shape needs ~134 MB of split partials: more than the
-    fixed array holds, so the call must refuse before launching anything."""
+    """1024 sequences with top-2048 need ~134 MB of candidate lists for just
+    one block of queries per sequence: more than the fixed array holds even
+    when run in chunks, so the call must refuse before launching anything."""
     a = lib.CsaArgs()
-    a.B, a.S, a.T, a.H_I, a.d, a.m, a.topk = 32, 64, 131072, 64, 128, 4, 2048
+    a.B, a.S, a.T, a.H_I, a.d, a.m, a.topk = 1024, 4, 8192, 64, 128, 4, 2048
     a.causal, a.q_offset = 1, -1
     a.q = a.w = a.k = a.out_idx = a.out_score = 1 << 20  # never dereferenced
     st = lib.csa_indexer_topk_noalloc(a, None)
