@@ -342,6 +342,13 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
         return CSA_ERR_CUDA;
 
     const KernelFn kern = pick_kernel(plan);
+    // The kernel's warpgroups trade registers (setmaxnreg); that only adds up
+    // when the kernel was built with exactly the launch count it assumes.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    if (fa.numRegs != csa::kLaunchRegs)
+        return CSA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes) !=
         cudaSuccess)
         return CSA_ERR_CUDA;

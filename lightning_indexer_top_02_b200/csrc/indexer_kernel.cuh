@@ -16,14 +16,18 @@
 // range; select_kernel.cuh turns the lists into the exact, sorted top k.  The
 // [B,S,H_I,T] score tensor never exists and the extra memory is O(S * k).
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: the query block once per item (with an L2
+// Warp roles (384 threads, three warpgroups):
+//   warps 0..3  epilogue warpgroup 0: the first half of the item's queries
+//   warps 4..7  epilogue warpgroup 1: the second half (idle when qps == 1)
+//   warp 8      TMA producer: the query block once per item (with an L2
 //               prefetch of the next item's), key tiles into a ring
-//   warp 1      TMEM owner and MMA issuer (one thread): per key tile, d/16
+//   warp 9      TMEM owner and MMA issuer (one thread): per key tile, d/16
 //               tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
 //               256-column TMEM accumulators
-//   warps 2..5  epilogue warpgroup 0: the first half of the item's queries
-//   warps 6..9  epilogue warpgroup 1: the second half (idle when qps == 1)
+//   warps 10,11 idle
+// The block launches with 168 registers per thread; the producer/MMA
+// warpgroup gives most of its share to the two epilogue warpgroups
+// (3 x 128 x 168 = 2 x 128 x kEpiRegs + 128 x kCtlRegs).
 //
 // Epilogue fast path (H_I >= 32, at most 128 TMEM columns per warpgroup): a
 // warp reads its 32 TMEM lanes with two 16-lane x 256-bit loads, so every
@@ -43,8 +47,12 @@ namespace csa {
 
 constexpr int kTileKeys = 128;   // MMA M: keys per tile
 constexpr int kSlotCols = 256;   // TMEM columns per accumulator slot
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;  // registers per thread the kernel must be built with
+constexpr int kEpiRegs = 224;     // after the split: epilogue warpgroups
+constexpr int kCtlRegs = 56;      //                  producer / MMA warpgroup
+static_assert(2 * 128 * kEpiRegs + 128 * kCtlRegs == kThreads * kLaunchRegs,
+              "register split must match the launch budget");
 constexpr int kGroupThreads = 128;
 constexpr int kBarWg0 = 1, kBarWg1 = 2;  // named barriers of the epilogue warpgroups
 constexpr int kEpt = 32;         // candidate keys per thread in a group (cap <= 4096)
@@ -354,10 +362,18 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
 {
     const int n = st.cnt;
     uint64_t e[kEpt];
+    // 16-byte loads: thread tid takes keys 2*(i*128 + tid) and the one after
 #pragma unroll
-    for (int i = 0; i < kEpt; ++i) {
-        const int j = i * kGroupThreads + tid;
-        e[i] = j < n ? list[j] : 0ull;
+    for (int i = 0; i < kEpt / 2; ++i) {
+        const int j = 2 * (i * kGroupThreads + tid);
+        if (j + 1 < n) {
+            const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(list + j);
+            e[2 * i] = v.x;
+            e[2 * i + 1] = v.y;
+        } else {
+            e[2 * i] = j < n ? list[j] : 0ull;
+            e[2 * i + 1] = 0ull;
+        }
     }
     uint32_t mn_all, mx_all;
     group_ord_range<kGroupThreads, kEpt>(e, &sc->gs, bar, tid, &mn_all, &mx_all);
@@ -369,10 +385,13 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
         for (int i = tid; i < kNbCompact; i += kGroupThreads)
             sc->hist[i] = 0;
         named_bar_sync(bar, kGroupThreads);
+        int bk[kEpt]; // each key's bucket, -1 for an empty slot
 #pragma unroll
-        for (int i = 0; i < kEpt; ++i)
-            if (e[i] != 0)
-                atomicAdd(&sc->hist[bucket_of_sqrt(key_score(e[i]), bm, kNbCompact)], 1u);
+        for (int i = 0; i < kEpt; ++i) {
+            bk[i] = e[i] != 0 ? bucket_of_sqrt(key_score(e[i]), bm, kNbCompact) : -1;
+            if (bk[i] >= 0)
+                atomicAdd(&sc->hist[bk[i]], 1u);
+        }
         named_bar_sync(bar, kGroupThreads);
         bucket_boundary<kGroupThreads, kNbCompact>(sc->hist, p.topk, false, &sc->gs, bar, tid);
         const int bstar = sc->gs.bcast[0];
@@ -384,7 +403,7 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
             uint32_t keep = 0;
 #pragma unroll
             for (int i = 0; i < kEpt; ++i) {
-                const bool k = e[i] != 0 && bucket_of_sqrt(key_score(e[i]), bm, kNbCompact) >= bstar;
+                const bool k = bk[i] >= bstar;
                 keep |= k ? (1u << i) : 0u;
                 mine += k ? 1 : 0;
                 mn = k ? min(mn, key_ord(e[i])) : mn;
@@ -459,7 +478,7 @@ template <> struct Ld16x256<128> {
 // queries: weight 2i+e belongs to column 8i + 2(lane%4) + e.
 template <int FC, int FQ>
 __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int j0, int lane,
-                                            float (&wr)[FC / 4])
+                                            float2 (&wr)[FC / 8])
 {
     constexpr int RPQ = FC / 8 / FQ;  // 8-column repetitions per query
 #pragma unroll
@@ -472,20 +491,24 @@ __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int
             a = src[0];
             b = src[1];
         }
-        wr[2 * i] = a;
-        wr[2 * i + 1] = b;
+        wr[i] = make_float2(a, b);
     }
+}
+
+__device__ __forceinline__ float2 relu2(uint32_t a, uint32_t b)
+{
+    return make_float2(fmaxf(__uint_as_float(a), 0.0f), fmaxf(__uint_as_float(b), 0.0f));
 }
 
 // Scores of FQ queries for one key per thread.  The warp's two 16-lane loads
 // cover its 32 keys; thread t holds columns 8i + 2(t%4) + {0,1} of keys
 // t/4 + {0, 8, 16, 24}.  After the loads land the accumulator slot is released
 // (one arrive per warp).  Each thread then forms per-key partial sums over its
-// columns; the quad (threads sharing t/4) exchanges halves twice so that
-// thread t ends with the complete scores of key row 16*((t>>1)&1) + 8*(t&1)
-// + t/4 of the warp's 32.
+// columns (column pairs with one packed FMA); the quad (threads sharing t/4)
+// exchanges halves twice so that thread t ends with the complete scores of
+// key row 16*((t>>1)&1) + 8*(t&1) + t/4 of the warp's 32.
 template <int FC, int FQ>
-__device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float (&wr)[FC / 4],
+__device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&wr)[FC / 8],
                                                  uint64_t *acc_empty, int lane, float (&F)[FQ])
 {
     constexpr int NV = FC / 2;
@@ -505,25 +528,21 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float (&w
     __syncwarp();
     if (lane == 0)
         mbar_arrive(acc_empty);
-    float P[4][FQ][2];
+    float2 P[4][FQ];
 #pragma unroll
     for (int k = 0; k < 4; ++k)
 #pragma unroll
         for (int j = 0; j < FQ; ++j)
-            P[k][j][0] = P[k][j][1] = 0.0f;
+            P[k][j] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int i = 0; i < REPS; ++i) {
         const int j = i / RPQ;
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float w = wr[2 * i + e];
-                P[sub][j][e] =
-                    fmaf(fmaxf(__uint_as_float(va[4 * i + 2 * sub + e]), 0.0f), w, P[sub][j][e]);
-                P[2 + sub][j][e] = fmaf(fmaxf(__uint_as_float(vb[4 * i + 2 * sub + e]), 0.0f), w,
-                                        P[2 + sub][j][e]);
-            }
+            P[sub][j] = __ffma2_rn(relu2(va[4 * i + 2 * sub], va[4 * i + 2 * sub + 1]), wr[i],
+                                   P[sub][j]);
+            P[2 + sub][j] = __ffma2_rn(relu2(vb[4 * i + 2 * sub], vb[4 * i + 2 * sub + 1]), wr[i],
+                                       P[2 + sub][j]);
         }
     }
     const bool b1 = (lane >> 1) & 1;
@@ -533,8 +552,8 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float (&w
         float R[2];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            const float lo = P[m][j][0] + P[m][j][1];          // key m (first 16 lanes)
-            const float hi = P[2 + m][j][0] + P[2 + m][j][1];  // key 2+m (last 16 lanes)
+            const float lo = P[m][j].x + P[m][j].y;          // key m (first 16 lanes)
+            const float hi = P[2 + m][j].x + P[2 + m][j].y;  // key 2+m (last 16 lanes)
             const float send = b1 ? lo : hi;
             const float keep = b1 ? hi : lo;
             R[m] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
@@ -542,6 +561,38 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float (&w
         const float send = b0 ? R[0] : R[1];
         const float keep = b0 ? R[1] : R[0];
         F[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+}
+
+// Appends this warp's surviving keys of FQ queries (one key per thread, the
+// queries' admission bounds and visibility ends cached in registers).
+template <int FQ>
+__device__ __forceinline__ void fast_emit(const float (&F)[FQ], const uint32_t (&bnd)[FQ],
+                                          const int (&vend)[FQ], int j0, int s, float kscale,
+                                          QueryState *qs, uint64_t *lbase, size_t lstride,
+                                          int lane)
+{
+    uint32_t ord[FQ];
+    unsigned bal[FQ];
+    int base[FQ];
+#pragma unroll
+    for (int q = 0; q < FQ; ++q) {
+        ord[q] = ord_of_score(F[q] * kscale);
+        bal[q] = __ballot_sync(0xffffffffu, s < vend[q] && ord[q] >= bnd[q]);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < FQ; ++q)
+            base[q] = bal[q] ? atomicAdd(&qs[j0 + q].cnt, __popc(bal[q])) : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < FQ; ++q) {
+        if (bal[q]) {
+            base[q] = __shfl_sync(0xffffffffu, base[q], 0);
+            if (bal[q] & (1u << lane))
+                lbase[static_cast<size_t>(j0 + q) * lstride + base[q] +
+                      __popc(bal[q] & lanemask_lt())] = make_key(ord[q], static_cast<uint32_t>(s));
+        }
     }
 }
 
@@ -576,7 +627,7 @@ template <int FC, int FQ, bool kHeadsGe32>
 __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uint32_t tmem_base,
                              const WaitCtl &ctl, int wg)
 {
-    const int tid = (threadIdx.x - 64) & (kGroupThreads - 1); // 0..127 within the warpgroup
+    const int tid = threadIdx.x & (kGroupThreads - 1); // 0..127 within the warpgroup
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int bar = wg == 0 ? kBarWg0 : kBarWg1;
@@ -616,7 +667,10 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                            : 0.0f;
         }
     }
-    float wr[FC > 0 ? FC / 4 : 1];
+    float2 wr[FC > 0 ? FC / 8 : 1];
+    constexpr int CQ = FC > 0 ? FQ : 1;
+    uint32_t bnd[CQ];   // fast path: this group's admission bounds and
+    int vend[CQ];       // visibility ends, cached from qs
 
     bool ok = true;
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
@@ -650,6 +704,13 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
             }
         }
         named_bar_sync(bar, kGroupThreads);
+        if constexpr (FC > 0) {
+#pragma unroll
+            for (int q = 0; q < CQ; ++q) {
+                bnd[q] = qs[j0 + q].bound;
+                vend[q] = qs[j0 + q].vis_end;
+            }
+        }
 
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
             const int s = t * kTileKeys + key_local;
@@ -671,7 +732,7 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                 if constexpr (FC > 0) {
                     float F[FQ];
                     fast_tile_scores<FC, FQ>(taddr, wr, &bars->acc_empty[slot], lane, F);
-                    emit_batch<FQ>(F, j0, s, kscale, qs, lbase, lstride, lane);
+                    fast_emit<FQ>(F, bnd, vend, j0, s, kscale, qs, lbase, lstride, lane);
                 } else {
                     // One chunk at a time, each query emitted as it completes.
                     auto emit = [&](int jq, float score) {
@@ -737,6 +798,11 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                     compact_list(p, lbase + static_cast<size_t>(jq) * lstride, qs[jq], sc, bar, tid);
                     pf.add(pa, kPfEpiCompact, rec);
                     pf.count(pa, kPfEpiCompactCount, rec);
+                    if constexpr (FC > 0) {
+#pragma unroll
+                        for (int q = 0; q < CQ; ++q)
+                            bnd[q] = qs[j0 + q].bound;
+                    }
                 }
             }
         }
@@ -785,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
     }
-    if (warp == 1) {
+    if (warp == 9) {
         tmem_alloc(&bars->tmem_addr, 2 * kSlotCols);
         tmem_relinquish();
     }
@@ -795,23 +861,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = bars->tmem_addr;
     WaitCtl ctl{&bars->abort, p.wait_limit};
 
-    if (warp == 0) {
-        if (lane == 0)
-            run_producer(p, &tmQ, &tmK, smem, bars, ctl);
-    } else if (warp == 1) {
-        if (lane == 0)
-            run_mma(p, smem, bars, tmem_base, ctl);
-    } else if (warp < 6) {
-        run_epilogue<FC, FQ, kHeadsGe32>(p, smem, bars, tmem_base, ctl, 0);
+    if (warp < 8) {
+        regs_inc<kEpiRegs>();
+        const int wg = warp >> 2;
+        if (wg < p.n_wg)
+            run_epilogue<FC, FQ, kHeadsGe32>(p, smem, bars, tmem_base, ctl, wg);
     } else {
-        if (p.n_wg == 2)
-            run_epilogue<FC, FQ, kHeadsGe32>(p, smem, bars, tmem_base, ctl, 1);
+        regs_dec<kCtlRegs>();
+        if (warp == 8 && lane == 0)
+            run_producer(p, &tmQ, &tmK, smem, bars, ctl);
+        else if (warp == 9 && lane == 0)
+            run_mma(p, smem, bars, tmem_base, ctl);
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) {
+    if (warp == 9) {
         __syncwarp();
         tmem_dealloc(tmem_base, 2 * kSlotCols);
     }

@@ -105,6 +105,22 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, con
     }
 }
 
+// ---------------------------------------------------------------- register split
+// Moves registers between warpgroups: every warp of a warpgroup executes the
+// same call.  An increase waits until enough registers have been released by
+// decreases, so the split must add up to what the block was launched with.
+template <int N>
+__device__ __forceinline__ void regs_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void regs_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 {
