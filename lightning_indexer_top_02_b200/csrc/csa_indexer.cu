@@ -381,7 +381,8 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
         sp.qb_lo = qb_lo;
         sp.out_idx = a->out_idx;
         sp.out_score = a->out_score;
-        const int sel_grid = sp.rows < 3 * sms ? sp.rows : 3 * sms;
+        const int sel_slots = csa::kSelCtasPerSm * sms;
+        const int sel_grid = sp.rows < sel_slots ? sp.rows : sel_slots;
         csa::select_topk_kernel<<<sel_grid, csa::kSelThreads, sel_smem, stream>>>(sp);
         if (cudaGetLastError() != cudaSuccess)
             return CSA_ERR_CUDA;

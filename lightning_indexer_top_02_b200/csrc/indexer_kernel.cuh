@@ -352,20 +352,74 @@ struct WgScratch {          // one per epilogue warpgroup
 };
 
 // ------------------------------------------------------------------ compaction
+// Bucket of the k-th largest key over a 1024-bucket histogram of the group:
+// {b*, keys in buckets above b*, keys in b*} with above < need <= above + in.
+// Thread tid owns buckets [8 tid, 8 tid + 8); two group barriers.
+__device__ __forceinline__ void compact_boundary(const uint32_t *hist, int need, GroupSmall *gs,
+                                                 int bar, int tid, int (&out)[3])
+{
+    constexpr int PER = kNbCompact / kGroupThreads;
+    const int lane = tid & 31, wid = tid >> 5;
+    uint32_t c[PER];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        c[j] = hist[tid * PER + j];
+        sum += c[j];
+    }
+    uint32_t suf = sum; // inclusive suffix sum over the warp's threads
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 32)
+            suf += t;
+    }
+    if (lane == 0)
+        gs->warp_sums[wid] = suf;
+    named_bar_sync(bar, kGroupThreads);
+    uint32_t higher = 0;
+#pragma unroll
+    for (int w = 0; w < kGroupThreads / 32; ++w)
+        higher += w > wid ? gs->warp_sums[w] : 0u;
+    const uint32_t above_thread = suf - sum + higher;
+    const uint32_t nd = static_cast<uint32_t>(need);
+    if (above_thread < nd && nd <= above_thread + sum) {
+        uint32_t above = above_thread;
+#pragma unroll
+        for (int j = PER - 1; j >= 0; --j) {
+            if (above + c[j] >= nd) {
+                gs->bcast[0] = tid * PER + j;
+                gs->bcast[1] = static_cast<int>(above);
+                gs->bcast[2] = static_cast<int>(c[j]);
+                break;
+            }
+            above += c[j];
+        }
+    }
+    named_bar_sync(bar, kGroupThreads);
+    out[0] = gs->bcast[0];
+    out[1] = gs->bcast[1];
+    out[2] = gs->bcast[2];
+}
+
 // Cuts a query's list back when it could overflow: keeps every key whose
-// bucket (over the list's own [min, max] score range) is at or above the
-// bucket of the k-th largest key -- a superset of the top k -- or, when the
-// range is degenerate or that bucket is too full, the radix-exact top k plus
-// slack.  Updates cnt and raises bound to the smallest kept score.
+// bucket is at or above the bucket of the k-th largest key -- a superset of
+// the top k -- or, when that bucket is too full, the radix-exact top k plus
+// slack.  Buckets split the list's own [min, max] range of score order images
+// into 1024 equal integer ranges.  Warp w owns list slots [1024 w, 1024 w +
+// 1024) (lane l: slots 1024 w + 64 i + 2 l and the one after) and writes the
+// keys it keeps back with coalesced stores.  Updates cnt and raises bound to
+// the smallest kept score.  The group's histogram is all zero on entry and on
+// return.
 __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, WgScratch *sc,
                              int bar, int tid)
 {
     const int n = st.cnt;
+    const int lane = tid & 31, wid = tid >> 5;
     uint64_t e[kEpt];
-    // 16-byte loads: thread tid takes keys 2*(i*128 + tid) and the one after
 #pragma unroll
     for (int i = 0; i < kEpt / 2; ++i) {
-        const int j = 2 * (i * kGroupThreads + tid);
+        const int j = wid * (kEpt * 32) + i * 64 + 2 * lane;
         if (j + 1 < n) {
             const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(list + j);
             e[2 * i] = v.x;
@@ -375,55 +429,89 @@ __device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, Wg
             e[2 * i + 1] = 0ull;
         }
     }
-    uint32_t mn_all, mx_all;
-    group_ord_range<kGroupThreads, kEpt>(e, &sc->gs, bar, tid, &mn_all, &mx_all);
-    const BucketMap bm = bucket_map_unit(mn_all, mx_all);
-    bool done = false;
-    uint32_t newmin = 0xFFFFFFFFu;
-    int kept = 0;
-    if (bm.ok) {
-        for (int i = tid; i < kNbCompact; i += kGroupThreads)
-            sc->hist[i] = 0;
-        named_bar_sync(bar, kGroupThreads);
-        int bk[kEpt]; // each key's bucket, -1 for an empty slot
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
 #pragma unroll
-        for (int i = 0; i < kEpt; ++i) {
-            bk[i] = e[i] != 0 ? bucket_of_sqrt(key_score(e[i]), bm, kNbCompact) : -1;
-            if (bk[i] >= 0)
-                atomicAdd(&sc->hist[bk[i]], 1u);
-        }
-        named_bar_sync(bar, kGroupThreads);
-        bucket_boundary<kGroupThreads, kNbCompact>(sc->hist, p.topk, false, &sc->gs, bar, tid);
-        const int bstar = sc->gs.bcast[0];
-        const int cand_kept = sc->gs.bcast[1] + sc->gs.bcast[2];
-        named_bar_sync(bar, kGroupThreads);
-        if (cand_kept <= p.cap - 2 * kTileKeys) {
-            int mine = 0;
-            uint32_t mn = 0xFFFFFFFFu;
-            uint32_t keep = 0;
-#pragma unroll
-            for (int i = 0; i < kEpt; ++i) {
-                const bool k = bk[i] >= bstar;
-                keep |= k ? (1u << i) : 0u;
-                mine += k ? 1 : 0;
-                mn = k ? min(mn, key_ord(e[i])) : mn;
-            }
-            int total;
-            int off = group_excl_scan<kGroupThreads>(mine, &sc->gs, bar, tid, &total);
-#pragma unroll
-            for (int i = 0; i < kEpt; ++i)
-                if (keep & (1u << i))
-                    list[off++] = e[i];
-            newmin = group_min_u32<kGroupThreads>(mn, &sc->gs, bar, tid);
-            kept = total;
-            done = true;
+    for (int i = 0; i < kEpt; ++i) {
+        if (e[i] != 0) {
+            lo = min(lo, key_ord(e[i]));
+            hi = max(hi, key_ord(e[i]));
         }
     }
-    if (!done) {
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+        sc->gs.warp_sums[wid] = lo;
+        sc->gs.warp_sums[16 + wid] = hi;
+    }
+    named_bar_sync(bar, kGroupThreads);
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+    for (int w = 0; w < kGroupThreads / 32; ++w) {
+        mn = min(mn, sc->gs.warp_sums[w]);
+        mx = max(mx, sc->gs.warp_sums[16 + w]);
+    }
+    const uint32_t span = mx - mn;
+    const int shift = span < static_cast<uint32_t>(kNbCompact) ? 0 : 32 - __clz(span) - 10;
+    int bk[kEpt]; // each key's bucket, -1 for an empty slot
+#pragma unroll
+    for (int i = 0; i < kEpt; ++i) {
+        bk[i] = e[i] != 0 ? static_cast<int>((key_ord(e[i]) - mn) >> shift) : -1;
+        if (bk[i] >= 0)
+            atomicAdd(&sc->hist[bk[i]], 1u);
+    }
+    named_bar_sync(bar, kGroupThreads);
+    int bd[3];
+    compact_boundary(sc->hist, p.topk, &sc->gs, bar, tid, bd);
+    // every thread read its own buckets in compact_boundary: clear them
+#pragma unroll
+    for (int j = 0; j < kNbCompact / kGroupThreads; ++j)
+        sc->hist[tid * (kNbCompact / kGroupThreads) + j] = 0;
+    const int bstar = bd[0];
+    const int cand_kept = bd[1] + bd[2];
+    uint32_t newmin = 0xFFFFFFFFu;
+    int kept = 0;
+    if (cand_kept <= p.cap - 2 * kTileKeys) {
+        uint32_t keep = 0;
+        int mine = 0;
+        uint32_t kmin = 0xFFFFFFFFu;
+#pragma unroll
+        for (int i = 0; i < kEpt; ++i) {
+            const bool k = bk[i] >= bstar;
+            keep |= k ? (1u << i) : 0u;
+            mine += k ? 1 : 0;
+            kmin = k ? min(kmin, key_ord(e[i])) : kmin;
+        }
+        const int wcount = __reduce_add_sync(0xffffffffu, mine);
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        if (lane == 0) {
+            sc->gs.warp_sums[wid] = static_cast<uint32_t>(wcount);
+            sc->gs.warp_sums[16 + wid] = kmin;
+        }
+        named_bar_sync(bar, kGroupThreads);
+        int pos = 0;
+#pragma unroll
+        for (int w = 0; w < kGroupThreads / 32; ++w) {
+            const int c = static_cast<int>(sc->gs.warp_sums[w]);
+            pos += w < wid ? c : 0;
+            kept += c;
+            newmin = min(newmin, sc->gs.warp_sums[16 + w]);
+        }
+        const unsigned lt = lanemask_lt();
+#pragma unroll
+        for (int i = 0; i < kEpt; ++i) {
+            const bool k = (keep >> i) & 1u;
+            const unsigned m = __ballot_sync(0xffffffffu, k);
+            if (k)
+                list[pos + __popc(m & lt)] = e[i];
+            pos += __popc(m);
+        }
+    } else {
         int k2;
         const uint64_t L = radix_bound<kGroupThreads, kEpt>(e, p.topk, p.slack, sc->hist, &sc->gs,
                                                             bar, tid, &k2);
         kept = write_kept<kGroupThreads, kEpt>(e, L, list, &sc->gs, bar, tid, &newmin);
+        for (int i = tid; i < kNbCompact; i += kGroupThreads)
+            sc->hist[i] = 0;
     }
     named_bar_sync(bar, kGroupThreads); // list writes and scratch reads done
     if (tid == 0) {
@@ -671,6 +759,10 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
     constexpr int CQ = FC > 0 ? FQ : 1;
     uint32_t bnd[CQ];   // fast path: this group's admission bounds and
     int vend[CQ];       // visibility ends, cached from qs
+
+    for (int i = tid; i < kNbCompact; i += kGroupThreads)
+        sc->hist[i] = 0;
+    named_bar_sync(bar, kGroupThreads);
 
     bool ok = true;
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {

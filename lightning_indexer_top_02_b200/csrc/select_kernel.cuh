@@ -9,19 +9,21 @@
 // query's lists holds its global top k.  Ranking: larger score first, equal
 // scores by lower key index (one comparison of the 64-bit keys).
 //
-// One CTA per query row at a time:
-//   1. If the lists hold more keys than fit in shared memory, a radix select
-//      over the 64-bit keys, reading them from global memory one byte per
-//      pass, finds the k-th largest key L; the k keys >= L are gathered.
-//      Otherwise every key is copied to shared memory.
-//   2. A histogram over NB buckets linear in the score, spanning the keys'
-//      own [min, max], finds the bucket holding the k-th largest key; the keys
-//      of that bucket and above are scattered into bucket order (a counting
-//      sort), and each bucket is then sorted on its own (insertion sort; the
-//      buckets average a few keys).  A bucket too full for that -- many equal
-//      or near-equal scores -- sends the row to a bitonic sort instead.
+// One CTA of 256 threads per query row at a time, several CTAs per SM:
+//   1. The row's keys go to registers (16 per thread).  Lists longer than
+//      that in total first go through a radix select over the 64-bit keys,
+//      read from global memory one byte per pass, which finds the k-th largest
+//      key L; the k keys >= L are gathered.
+//   2. A histogram over NB buckets linear in the score, spanning the keys' own
+//      [min, max], finds the bucket holding the k-th largest key; the keys of
+//      that bucket and above are scattered into bucket order (a counting
+//      sort); each key is then ranked among the keys of its own bucket and
+//      moved to its final slot (the buckets average a few keys).  A bucket too
+//      full for that -- many equal or near-equal scores -- sends the row to a
+//      bitonic sort instead.
 //   3. The first min(k, n) keys become (index, score) pairs; the rest of the
 //      row is padded with (-1, -inf).
+// While a row is processed, the next row's list is prefetched into L2.
 #pragma once
 #include <cstdint>
 
@@ -30,10 +32,11 @@
 
 namespace csa {
 
-constexpr int kSelThreads = 512;
-constexpr int kSelNb = 2048;          // histogram buckets
-constexpr int kSelKeys = 4096;        // keys held in shared memory
-constexpr int kSelSmallBucket = 24;   // largest bucket sorted by one thread
+constexpr int kSelThreads = 256;
+constexpr int kSelEpt = 16;                       // keys per thread in registers
+constexpr int kSelKeys = kSelThreads * kSelEpt;   // 4096
+constexpr int kSelNb = 2048;                      // histogram buckets
+constexpr int kSelSmallBucket = 64;               // largest bucket ordered by ranking
 constexpr int kSelMaxSplits = 64;
 
 struct SelParams {
@@ -52,43 +55,21 @@ struct SelSmem {
     int split_off[kSelMaxSplits + 1];
     int misc[4];
     uint32_t hist[kSelNb];
-    uint64_t in[kSelKeys];
     uint64_t out[kSelKeys];
+    uint64_t top[kMaxTopk];   // the sorted top k (fast path)
 };
 
-// Block-wide min and max of the score order images of a[0..n).
-__device__ __forceinline__ void sel_ord_range(const uint64_t *a, int n, GroupSmall *gs, int tid,
-                                              uint32_t *mn, uint32_t *mx)
+__device__ __forceinline__ void sel_prefetch_l2(const void *src, uint32_t bytes)
 {
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (int i = tid; i < n; i += kSelThreads) {
-        const uint32_t o = key_ord(a[i]);
-        lo = min(lo, o);
-        hi = max(hi, o);
-    }
-    lo = __reduce_min_sync(0xffffffffu, lo);
-    hi = __reduce_max_sync(0xffffffffu, hi);
-    const int lane = tid & 31, wid = tid >> 5;
-    if (lane == 0) {
-        gs->warp_sums[wid] = lo;
-        gs->warp_sums[16 + wid] = hi;
-    }
-    __syncthreads();
-    uint32_t a0 = 0xFFFFFFFFu, b0 = 0u;
-#pragma unroll
-    for (int w = 0; w < kSelThreads / 32; ++w) {
-        a0 = min(a0, gs->warp_sums[w]);
-        b0 = max(b0, gs->warp_sums[16 + w]);
-    }
-    __syncthreads();
-    *mn = a0;
-    *mx = b0;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(bytes)
+                 : "memory");
 }
 
 // Radix select over the row's lists in global memory: the largest L such that
 // exactly `need` keys are >= L (keys are distinct and non-zero; n > need).
-__device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_lists,
-                                     const SelSmem *ro, SelSmem *sm, int need, int tid)
+__device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_lists, SelSmem *sm,
+                                     int need, int tid)
 {
     const int lane = tid & 31;
     uint64_t prefix = 0, mask = 0;
@@ -98,7 +79,7 @@ __device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_li
         __syncthreads();
         for (int s = 0; s < sp.nsplit; ++s) {
             const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
-            const int n = ro->split_off[s + 1] - ro->split_off[s];
+            const int n = sm->split_off[s + 1] - sm->split_off[s];
             for (int j = tid; j < n; j += kSelThreads) {
                 const uint64_t x = src[j];
                 if ((x & mask) == prefix)
@@ -151,26 +132,51 @@ __device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_li
     return prefix;
 }
 
-// Sorts the keys of in[0..n) that belong to the top `kept` (kept <= n) into
-// descending order.  Returns the buffer holding them at [0, kept).
-__device__ uint64_t *sel_sort_top(SelSmem *sm, int n, int kept, int tid)
+// Sorts the n keys of e[] (0 = empty slot, n <= kSelKeys): returns a shared
+// buffer holding the top `kept` of them (kept <= n) in descending order at
+// [0, kept).
+__device__ const uint64_t *sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEpt], int n,
+                                         int kept, int tid)
 {
-    uint32_t mn, mx;
-    sel_ord_range(sm->in, n, &sm->gs, tid, &mn, &mx);
+    const int lane = tid & 31, wid = tid >> 5;
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+    for (int i = 0; i < kSelEpt; ++i) {
+        if (e[i] != 0) {
+            lo = min(lo, key_ord(e[i]));
+            hi = max(hi, key_ord(e[i]));
+        }
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+        sm->gs.warp_sums[wid] = lo;
+        sm->gs.warp_sums[16 + wid] = hi;
+    }
+    for (int i = tid; i < kSelNb; i += kSelThreads)
+        sm->hist[i] = 0;
+    __syncthreads();
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        mn = min(mn, sm->gs.warp_sums[w]);
+        mx = max(mx, sm->gs.warp_sums[16 + w]);
+    }
     const BucketMap bm = bucket_map(mn, mx, kSelNb);
-    bool fallback = !bm.ok;
     int total = n;
-    uint64_t *res = sm->in;
+    bool fallback = !bm.ok;
     if (!fallback) {
-        // histogram with buckets numbered from the top score down
-        for (int i = tid; i < kSelNb; i += kSelThreads)
-            sm->hist[i] = 0;
+        // histogram, buckets numbered from the top score down
+        int db[kSelEpt];
+#pragma unroll
+        for (int i = 0; i < kSelEpt; ++i) {
+            db[i] = e[i] != 0 ? kSelNb - 1 - bucket_of(key_score(e[i]), bm, kSelNb) : kSelNb;
+            if (db[i] < kSelNb)
+                atomicAdd(&sm->hist[db[i]], 1u);
+        }
         __syncthreads();
-        for (int i = tid; i < n; i += kSelThreads)
-            atomicAdd(&sm->hist[kSelNb - 1 - bucket_of(key_score(sm->in[i]), bm, kSelNb)], 1u);
-        __syncthreads();
-        // exclusive prefix over buckets (top first): hist[b] becomes the first
-        // slot of bucket b; find the bucket db* holding slot kept-1
+        // exclusive prefix over buckets: hist[b] becomes the first slot of
+        // bucket b; find the bucket db* that holds slot kept-1
         constexpr int PER = kSelNb / kSelThreads;
         uint32_t c[PER];
         uint32_t sum = 0;
@@ -179,9 +185,20 @@ __device__ uint64_t *sel_sort_top(SelSmem *sm, int n, int kept, int tid)
             c[j] = sm->hist[tid * PER + j];
             sum += c[j];
         }
-        int tot;
-        const int base = group_excl_scan<kSelThreads>(static_cast<int>(sum), &sm->gs, 0, tid, &tot);
-        uint32_t run = static_cast<uint32_t>(base);
+        uint32_t inc = sum; // inclusive prefix over the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off)
+                inc += t;
+        }
+        if (lane == 31)
+            sm->gs.warp_sums[wid] = inc; // the min/max reads finished before the last barrier
+        __syncthreads();
+        uint32_t run = inc - sum;
+#pragma unroll
+        for (int w = 0; w < kSelThreads / 32; ++w)
+            run += w < wid ? sm->gs.warp_sums[w] : 0u;
         int biggest = 0;
 #pragma unroll
         for (int j = 0; j < PER; ++j) {
@@ -189,15 +206,16 @@ __device__ uint64_t *sel_sort_top(SelSmem *sm, int n, int kept, int tid)
             sm->hist[tid * PER + j] = start;
             run += c[j];
             if (start < static_cast<uint32_t>(kept) && run >= static_cast<uint32_t>(kept)) {
-                sm->misc[0] = tid * PER + j;   // db*
-                sm->misc[1] = static_cast<int>(run); // keys in buckets <= db*
+                sm->misc[0] = tid * PER + j;          // db*
+                sm->misc[1] = static_cast<int>(run);  // keys in buckets <= db*
             }
             if (start < static_cast<uint32_t>(kept))
                 biggest = max(biggest, static_cast<int>(c[j]));
         }
         biggest = __reduce_max_sync(0xffffffffu, biggest);
-        if ((tid & 31) == 0)
-            sm->gs.warp_sums[tid >> 5] = static_cast<uint32_t>(biggest);
+        __syncthreads(); // warp_sums reads done
+        if (lane == 0)
+            sm->gs.warp_sums[wid] = static_cast<uint32_t>(biggest);
         __syncthreads();
         const int dstar = sm->misc[0];
         total = sm->misc[1];
@@ -205,48 +223,57 @@ __device__ uint64_t *sel_sort_top(SelSmem *sm, int n, int kept, int tid)
 #pragma unroll
         for (int w = 0; w < kSelThreads / 32; ++w)
             big = max(big, static_cast<int>(sm->gs.warp_sums[w]));
-        __syncthreads();
         // scatter the keys of buckets <= db* into bucket order
-        for (int i = tid; i < n; i += kSelThreads) {
-            const uint64_t x = sm->in[i];
-            const int db = kSelNb - 1 - bucket_of(key_score(x), bm, kSelNb);
-            if (db <= dstar)
-                sm->out[atomicAdd(&sm->hist[db], 1u)] = x;
-        }
+#pragma unroll
+        for (int i = 0; i < kSelEpt; ++i)
+            if (db[i] <= dstar)
+                sm->out[atomicAdd(&sm->hist[db[i]], 1u)] = e[i];
         __syncthreads();
-        res = sm->out;
-        if (big > kSelSmallBucket) {
-            fallback = true;
-        } else {
-            // bucket db now spans [end(db-1), end(db)) where end = hist after the scatter
-            for (int db = tid; db <= dstar; db += kSelThreads) {
-                const int lo = db == 0 ? 0 : static_cast<int>(sm->hist[db - 1]);
-                const int hi = static_cast<int>(sm->hist[db]);
-                for (int a = lo + 1; a < hi; ++a) {
-                    const uint64_t x = sm->out[a];
-                    int b = a - 1;
-                    while (b >= lo && sm->out[b] < x) {
-                        sm->out[b + 1] = sm->out[b];
-                        --b;
-                    }
-                    sm->out[b + 1] = x;
-                }
+        if (big <= kSelSmallBucket) {
+            // Rank each placed key inside its bucket (keys are distinct) and
+            // write it to bucket start + rank when that slot is among the
+            // first `kept`.  Keys go to threads in slot order, so the lanes of
+            // a warp see buckets of similar size.
+            for (int a = tid; a < total; a += kSelThreads) {
+                const uint64_t x = sm->out[a];
+                const int b = kSelNb - 1 - bucket_of(key_score(x), bm, kSelNb);
+                const int lo_s = b == 0 ? 0 : static_cast<int>(sm->hist[b - 1]);
+                const int hi_s = static_cast<int>(sm->hist[b]);
+                int to = lo_s;
+                for (int j = lo_s; j < hi_s; ++j)
+                    to += sm->out[j] > x ? 1 : 0;
+                if (to < kept)
+                    sm->top[to] = x;
             }
             __syncthreads();
+            return sm->top;
         }
+    } else {
+        // degenerate range (one score for every key): all keys to out[]
+        int mine = 0;
+#pragma unroll
+        for (int i = 0; i < kSelEpt; ++i)
+            mine += e[i] != 0;
+        int tot;
+        int off = group_excl_scan<kSelThreads>(mine, &sm->gs, 0, tid, &tot);
+#pragma unroll
+        for (int i = 0; i < kSelEpt; ++i)
+            if (e[i] != 0)
+                sm->out[off++] = e[i];
+        total = tot;
     }
-    if (fallback) {
-        // bitonic sort of res[0..total) padded with empty keys to a power of two
-        const int P = pow2_at_least(total);
-        for (int i = total + tid; i < P; i += kSelThreads)
-            res[i] = 0ull;
-        __syncthreads();
-        bitonic_sort_desc<kSelThreads>(res, P, 0, tid);
-    }
-    return res;
+    // bitonic sort of out[0..total) padded with empty keys to a power of two
+    const int P = pow2_at_least(total);
+    for (int i = total + tid; i < P; i += kSelThreads)
+        sm->out[i] = 0ull;
+    __syncthreads();
+    bitonic_sort_desc<kSelThreads>(sm->out, P, 0, tid);
+    return sm->out;
 }
 
-__global__ void __launch_bounds__(kSelThreads)
+constexpr int kSelCtasPerSm = 3;
+
+__global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
     select_topk_kernel(const SelParams sp)
 {
     extern __shared__ uint8_t sel_smem_raw[];
@@ -261,19 +288,46 @@ __global__ void __launch_bounds__(kSelThreads)
             continue;
         const size_t orow = static_cast<size_t>(b) * sp.S + q;
         const uint64_t *row_lists = sp.lists + static_cast<size_t>(r) * sp.nsplit * sp.cap;
-        if (tid == 0) {
-            int off = 0;
-            sm->split_off[0] = 0;
-            for (int s = 0; s < sp.nsplit; ++s) {
-                off += sp.counts[static_cast<size_t>(r) * sp.nsplit + s];
-                sm->split_off[s + 1] = off;
+        if (tid < 32) {
+            // list lengths -> offsets (nsplit <= 64: two per lane)
+            const int lane = tid;
+            const int c0 = lane < sp.nsplit ? sp.counts[static_cast<size_t>(r) * sp.nsplit + lane] : 0;
+            const int c1 = lane + 32 < sp.nsplit
+                               ? sp.counts[static_cast<size_t>(r) * sp.nsplit + lane + 32]
+                               : 0;
+            int x0 = c0, x1 = c1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int t0 = __shfl_up_sync(0xffffffffu, x0, off);
+                const int t1 = __shfl_up_sync(0xffffffffu, x1, off);
+                if (lane >= off) {
+                    x0 += t0;
+                    x1 += t1;
+                }
+            }
+            const int tot0 = __shfl_sync(0xffffffffu, x0, 31);
+            if (lane == 0)
+                sm->split_off[0] = 0;
+            if (lane < sp.nsplit)
+                sm->split_off[lane + 1] = x0;
+            if (lane + 32 < sp.nsplit)
+                sm->split_off[lane + 33] = tot0 + x1;
+        } else if (tid == 32) {
+            // warm L2 with the next row's first list
+            const int rn = r + gridDim.x;
+            if (rn < sp.rows) {
+                const int cn = sp.counts[static_cast<size_t>(rn) * sp.nsplit];
+                const uint32_t bytes = static_cast<uint32_t>((cn * 8 + 15) & ~15);
+                if (bytes > 0)
+                    sel_prefetch_l2(sp.lists + static_cast<size_t>(rn) * sp.nsplit * sp.cap, bytes);
             }
         }
         __syncthreads();
         const int n_all = sm->split_off[sp.nsplit];
         int n = n_all;
+        uint64_t e[kSelEpt];
         if (n_all > kSelKeys) {
-            const uint64_t L = sel_radix_global(sp, row_lists, sm, sm, sp.topk, tid);
+            const uint64_t L = sel_radix_global(sp, row_lists, sm, sp.topk, tid);
             if (tid == 0)
                 sm->misc[2] = 0;
             __syncthreads();
@@ -283,22 +337,41 @@ __global__ void __launch_bounds__(kSelThreads)
                 for (int j = tid; j < ns; j += kSelThreads) {
                     const uint64_t x = src[j];
                     if (x >= L)
-                        sm->in[atomicAdd(&sm->misc[2], 1)] = x;
+                        sm->out[atomicAdd(&sm->misc[2], 1)] = x;
                 }
             }
+            __syncthreads();
             n = sp.topk;
+#pragma unroll
+            for (int i = 0; i < kSelEpt; ++i) {
+                const int j = i * kSelThreads + tid;
+                e[i] = j < n ? sm->out[j] : 0ull;
+            }
+            __syncthreads(); // out[] is rewritten below
+        } else if (sp.nsplit == 1) {
+#pragma unroll
+            for (int i = 0; i < kSelEpt; ++i) {
+                const int j = i * kSelThreads + tid;
+                e[i] = j < n ? row_lists[j] : 0ull;
+            }
         } else {
             for (int s = 0; s < sp.nsplit; ++s) {
                 const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
                 const int o = sm->split_off[s];
                 const int ns = sm->split_off[s + 1] - o;
                 for (int j = tid; j < ns; j += kSelThreads)
-                    sm->in[o + j] = src[j];
+                    sm->out[o + j] = src[j];
             }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < kSelEpt; ++i) {
+                const int j = i * kSelThreads + tid;
+                e[i] = j < n ? sm->out[j] : 0ull;
+            }
+            __syncthreads(); // out[] is rewritten below
         }
-        __syncthreads();
         const int kept = min(n, sp.topk);
-        const uint64_t *res = kept > 0 ? sel_sort_top(sm, n, kept, tid) : sm->in;
+        const uint64_t *res = kept > 0 ? sel_sort_regs(sm, e, n, kept, tid) : sm->out;
         int32_t *oi = sp.out_idx + orow * sp.topk;
         float *os = sp.out_score + orow * sp.topk;
         for (int i = tid; i < sp.topk; i += kSelThreads) {
