@@ -2,8 +2,10 @@
 """Benchmark of the CSA lightning-indexer top-k on B200.
 
 One step = one call of the C-ABI entry point over one batch of synthetic
-inputs resident in HBM (the fused indexer/top-k kernel, plus the split merge
-when the plan splits key ranges).  Prints ONE JSON line on rank 0.
+inputs resident in HBM: the fused scoring/candidate-filter kernel and the
+exact top-k select over its candidate lists.  Prints ONE JSON line on rank 0.
+The roofline figure is the fused kernel's own duration, taken from CUDA
+events the library records around its launches (csa_set_launch_events).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
                     [--impl reference]
@@ -44,6 +46,35 @@ def load_peaks():
         return d, "measured"
     except OSError:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sources_sha() -> str:
+    """Hash of the CUDA sources: a traffic figure measured on other sources is stale."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for path in sorted(glob.glob(os.path.join(ROOT, "lightning_indexer_top_02_b200", "csrc", "*"))):
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(config: str, sha: str):
+    """DRAM bytes per fused-kernel launch from profiles/traffic.txt (ncu
+    dram__bytes_read.sum + dram__bytes_write.sum), or None when no capture of
+    these exact sources and this workload is recorded."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 4 and not line.startswith("#") and parts[0] == config \
+                        and parts[2] == sha:
+                    return int(parts[3])
+    except OSError:
+        pass
+    return None
 
 
 def dist_env():
@@ -248,6 +279,14 @@ def main():
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # events around each kernel launch of each step (fused, select, end)
+    n_marks = plan.launches + 1
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)]
+             for _ in range(args.steps)]
+    for row in marks:
+        for e in row:
+            e.record(stream)  # creates the event
+    torch.cuda.synchronize(dev)
     sampler = None
     if rank == 0:
         props = torch.cuda.get_device_properties(dev)
@@ -260,9 +299,11 @@ def main():
     torch.cuda.synchronize(dev)
     for i in range(args.steps):
         flush.zero_()
+        L.csa_set_launch_events(marks[i])
         starts[i].record(stream)
         step()
         ends[i].record(stream)
+    L.csa_set_launch_events(None)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -270,6 +311,11 @@ def main():
     if L.csa_last_device_error(sptr) != L.CSA_OK:
         raise SystemExit("device error during the timed region")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    # per launch chunk: fused kernel between marks 2c and 2c+1, select between 2c+1 and 2c+2
+    fused_ms = [sum(row[2 * c].elapsed_time(row[2 * c + 1]) for c in range(plan.launches // 2))
+                for row in marks]
+    select_ms = [sum(row[2 * c + 1].elapsed_time(row[2 * c + 2])
+                     for c in range(plan.launches // 2)) for row in marks]
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -336,11 +382,16 @@ def main():
     timed_s = total_ms / 1000.0
     sustained = timed_s > 0.5
     peak = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
-    roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                "frac": tflops / peak if peak else None, "traffic": None,
+    fused_avg = statistics.mean(fused_ms)
+    k_tflops = flops / (fused_avg / 1000.0) / 1e12
+    sha = kernel_sources_sha()
+    roofline = {"bound": "tensor", "achieved": k_tflops, "peak": peak, "unit": "TFLOP/s",
+                "frac": k_tflops / peak if peak else None,
+                "traffic": measured_traffic(wl.name, sha),
                 "peak_source": f"{peak_src} bf16 dense ({'sustained' if sustained else 'burst'})",
-                "kernel": "indexer_topk_kernel (+ split merge when the plan splits)",
-                "algorithmic_flops_per_launch": flops}
+                "kernel": "indexer_topk_kernel (fused scoring + candidate filter)",
+                "kernel_ms": fused_avg, "select_kernel_ms": statistics.mean(select_ms),
+                "algorithmic_flops_per_launch": flops, "sources_sha": sha}
     cpu = None
     if not args.no_cpu_baseline:
         cpu_inputs = inputs_for_oracle(wl, {"q": q, "w": w, "k": k, "k_scale": ks})

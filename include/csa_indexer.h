@@ -144,7 +144,9 @@ typedef struct {
     int stages;            /* key-tile pipeline depth                            */
     int queries_per_block; /* queries one work item covers                       */
     int num_splits;        /* key-range splits per query block                   */
-    int launches;          /* kernel launches per call (1, or 2 with a merge)    */
+    int launches;          /* kernel launches per call: per launch chunk the      *
+                            * fused scoring/filter kernel and the exact top-k   *
+                            * select (0 or 1 for the empty cases)               */
     size_t workspace_bytes;
 } csa_plan_t;
 
@@ -173,6 +175,19 @@ csa_status_t csa_last_device_error(cudaStream_t stream);
  * Tests shrink it to make a wait run out on purpose.  0 restores the default.
  */
 void csa_set_wait_limit(unsigned long long cycles);
+
+/*
+ * Measurement hook (no counterpart in the pages): while set, every later call
+ * on this host thread records events[j] on its stream immediately before its
+ * j-th kernel launch and events[L] after its last one (L = launches of the
+ * call), for j < n; events beyond n are not recorded.  For a single-chunk
+ * plan the fused kernel runs between events[0] and events[1] and the top-k
+ * select between events[1] and events[2].  The caller owns the events
+ * (created with timing enabled) and keeps them alive while set; pass
+ * (NULL, 0) to stop.  Returns CSA_ERR_INVALID_ARG for n < 0 or a NULL array
+ * with n > 0.
+ */
+csa_status_t csa_set_launch_events(cudaEvent_t *events, int n);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int csa_version(void);

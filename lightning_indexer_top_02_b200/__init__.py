@@ -8,7 +8,8 @@ functions below raises.
 
 C-ABI names are mirrored one to one (``csa_indexer_topk``,
 ``csa_indexer_topk_ex``, ``csa_indexer_workspace_size``, ``csa_status_string``,
-``csa_last_device_error``, ``csa_set_wait_limit``, ``csa_version``);
+``csa_last_device_error``, ``csa_set_wait_limit``, ``csa_set_launch_events``,
+``csa_version``);
 ``indexer_topk`` is the same call on torch tensors.
 """
 from __future__ import annotations
@@ -32,7 +33,8 @@ CSA_MODE_GATE = 1
 
 EXPORTS = ("csa_indexer_topk", "csa_indexer_topk_ex", "csa_indexer_workspace_size",
            "csa_indexer_plan", "csa_indexer_topk_noalloc", "csa_status_string",
-           "csa_last_device_error", "csa_set_wait_limit", "csa_version")
+           "csa_last_device_error", "csa_set_wait_limit", "csa_set_launch_events",
+           "csa_version")
 
 
 class CsaError(RuntimeError):
@@ -92,6 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.csa_last_device_error.restype = I
     lib.csa_set_wait_limit.argtypes = [ctypes.c_ulonglong]
     lib.csa_set_wait_limit.restype = None
+    lib.csa_set_launch_events.argtypes = [P, I]
+    lib.csa_set_launch_events.restype = I
     lib.csa_version.argtypes = []
     lib.csa_version.restype = I
     _lib = lib
@@ -138,6 +142,22 @@ def csa_last_device_error(stream_ptr=None) -> int:
 
 def csa_set_wait_limit(cycles: int) -> None:
     load_library().csa_set_wait_limit(cycles)
+
+
+def csa_set_launch_events(events) -> int:
+    """Record ``events`` (torch.cuda.Event with timing, or raw cudaEvent_t
+    handles) around every kernel launch of later calls on this thread; pass
+    None or [] to stop.  The list must stay alive while set."""
+    global _event_array
+    if not events:
+        _event_array = None
+        return load_library().csa_set_launch_events(None, 0)
+    handles = [e.cuda_event if hasattr(e, "cuda_event") else int(e) for e in events]
+    _event_array = (ctypes.c_void_p * len(handles))(*handles)
+    return load_library().csa_set_launch_events(_event_array, len(handles))
+
+
+_event_array = None
 
 
 def csa_version() -> int:

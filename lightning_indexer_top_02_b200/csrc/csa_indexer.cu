@@ -25,6 +25,18 @@ constexpr unsigned long long kDefaultWaitLimit = 4000000000ull;
 
 unsigned long long g_wait_limit = kDefaultWaitLimit;
 
+// Measurement hook: events recorded around this thread's launches.
+thread_local cudaEvent_t *t_events = nullptr;
+thread_local int t_n_events = 0;
+
+// Records event j of the current call, if the caller asked for it.
+bool mark(int j, cudaStream_t stream)
+{
+    if (j >= t_n_events)
+        return true;
+    return cudaEventRecord(t_events[j], stream) == cudaSuccess;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -101,8 +113,6 @@ csa_status_t validate(const csa_args_t *a)
         return CSA_ERR_UNSUPPORTED;
     if (a->topk > csa::kMaxTopk)
         return CSA_ERR_UNSUPPORTED;
-    if (a->key_dtype == CSA_KEY_E4M3)
-        return CSA_ERR_UNSUPPORTED; // FP8 keys: not yet built
     const long long rows_q = static_cast<long long>(a->B) * a->S * a->H_I;
     const long long rows_k = static_cast<long long>(a->B) * a->T;
     if (rows_q >= (1ll << 31) || rows_k >= (1ll << 31))
@@ -178,7 +188,9 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
         return CSA_ERR_UNSUPPORTED;
     p.slack = (p.cap - csa::kTileKeys - p.topk) / 2;
 
-    const int k_stage = csa::kTileKeys * p.d * 2;
+    // per pipeline stage: the MMA's 16-bit key tile, plus (E4M3 keys) the raw
+    // staged tile it is converted from
+    const int k_stage = csa::kTileKeys * p.d * 2 + (p.key_fp8 ? csa::kTileKeys * p.d : 0);
     int off = 0;
     p.off_q = off;
     off += p.N * p.d * 2;
@@ -196,7 +208,10 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     if (stages < 2)
         return CSA_ERR_UNSUPPORTED;
     p.stages = stages;
-    off += stages * k_stage;
+    off += stages * csa::kTileKeys * p.d * 2;
+    p.off_k8 = off;
+    if (p.key_fp8)
+        off += stages * csa::kTileKeys * p.d;
     p.off_w = off;
     off += p.qps * p.H * 4;
     off = (off + 15) / 16 * 16;
@@ -281,13 +296,13 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
 }
 
 bool make_tmap(CUtensorMap *tm, CUtensorMapDataType dt, const void *base, long long rows, int cols,
-               int box_cols, int box_rows, CUtensorMapSwizzle swz)
+               int box_cols, int box_rows, CUtensorMapSwizzle swz, int elem_bytes = 2)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
         return false;
     const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estride[2] = {1, 1};
     return enc(tm, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
@@ -337,9 +352,15 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
     if (!make_tmap(&tmQ, qdt, a->q, static_cast<long long>(p.B) * p.S * p.H, p.d, p.row_bytes / 2,
                    p.N, swz))
         return CSA_ERR_CUDA;
-    if (!make_tmap(&tmK, qdt, a->k, static_cast<long long>(p.B) * p.T, p.d, p.row_bytes / 2,
-                   csa::kTileKeys, swz))
+    if (p.key_fp8) {
+        // raw E4M3 rows, unswizzled: the converters rewrite them swizzled
+        if (!make_tmap(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->k, static_cast<long long>(p.B) * p.T,
+                       p.d, p.d, csa::kTileKeys, CU_TENSOR_MAP_SWIZZLE_NONE, 1))
+            return CSA_ERR_CUDA;
+    } else if (!make_tmap(&tmK, qdt, a->k, static_cast<long long>(p.B) * p.T, p.d,
+                          p.row_bytes / 2, csa::kTileKeys, swz)) {
         return CSA_ERR_CUDA;
+    }
 
     const KernelFn kern = pick_kernel(plan);
     // The kernel's warpgroups trade registers (setmaxnreg); that only adds up
@@ -357,6 +378,7 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
                              sel_smem) != cudaSuccess)
         return CSA_ERR_CUDA;
     const int sms = device_sms();
+    int launched = 0;
     for (int qb_lo = 0; qb_lo < plan.nqb_total; qb_lo += plan.qb_chunk) {
         const int nqb = plan.nqb_total - qb_lo < plan.qb_chunk ? plan.nqb_total - qb_lo
                                                               : plan.qb_chunk;
@@ -364,6 +386,8 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
         p.nqb = nqb;
         p.n_items = p.B * nqb * p.nsplit;
         const int grid = p.n_items < plan.grid ? p.n_items : plan.grid;
+        if (!mark(launched++, stream))
+            return CSA_ERR_CUDA;
         kern<<<grid, csa::kThreads, p.smem_bytes, stream>>>(tmQ, tmK, p);
         if (cudaGetLastError() != cudaSuccess)
             return CSA_ERR_CUDA;
@@ -383,10 +407,14 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
         sp.out_score = a->out_score;
         const int sel_slots = csa::kSelCtasPerSm * sms;
         const int sel_grid = sp.rows < sel_slots ? sp.rows : sel_slots;
+        if (!mark(launched++, stream))
+            return CSA_ERR_CUDA;
         csa::select_topk_kernel<<<sel_grid, csa::kSelThreads, sel_smem, stream>>>(sp);
         if (cudaGetLastError() != cudaSuccess)
             return CSA_ERR_CUDA;
     }
+    if (!mark(launched, stream))
+        return CSA_ERR_CUDA;
     return CSA_OK;
 }
 
@@ -536,6 +564,15 @@ csa_status_t csa_last_device_error(cudaStream_t stream)
 void csa_set_wait_limit(unsigned long long cycles)
 {
     g_wait_limit = cycles ? cycles : kDefaultWaitLimit;
+}
+
+csa_status_t csa_set_launch_events(cudaEvent_t *events, int n)
+{
+    if (n < 0 || (n > 0 && !events))
+        return CSA_ERR_INVALID_ARG;
+    t_events = n > 0 ? events : nullptr;
+    t_n_events = n;
+    return CSA_OK;
 }
 
 int csa_version(void) { return kVersion; }

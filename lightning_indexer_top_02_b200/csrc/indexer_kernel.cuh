@@ -24,7 +24,13 @@
 //   warp 9      TMEM owner and MMA issuer (one thread): per key tile, d/16
 //               tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
 //               256-column TMEM accumulators
-//   warps 10,11 idle
+//   warps 10,11 E4M3 keys only: converters.  The producer lands each FP8 key
+//               tile in a staging ring; the converters rewrite it as f16
+//               into the MMA's swizzled key ring (exact: every E4M3 value is
+//               an f16 normal) and convert the item's query block from bf16
+//               to f16 in place (exact for |q| < 65504), so the MMA runs
+//               kind::f16 with both operands f16.  The key's fp32 scale
+//               multiplies its score after the head reduction (scale > 0).
 // The block launches with 168 registers per thread; the producer/MMA
 // warpgroup gives most of its share to the two epilogue warpgroups
 // (3 x 128 x 168 = 2 x 128 x kEpiRegs + 128 x kCtlRegs).
@@ -38,6 +44,8 @@
 // per thread with 32-lane loads and weights from shared memory.
 #pragma once
 #include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -49,8 +57,8 @@ constexpr int kTileKeys = 128;   // MMA M: keys per tile
 constexpr int kSlotCols = 256;   // TMEM columns per accumulator slot
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;  // registers per thread the kernel must be built with
-constexpr int kEpiRegs = 224;     // after the split: epilogue warpgroups
-constexpr int kCtlRegs = 56;      //                  producer / MMA warpgroup
+constexpr int kEpiRegs = 216;     // after the split: epilogue warpgroups
+constexpr int kCtlRegs = 72;      //                  producer / MMA warpgroup
 static_assert(2 * 128 * kEpiRegs + 128 * kCtlRegs == kThreads * kLaunchRegs,
               "register split must match the launch budget");
 constexpr int kGroupThreads = 128;
@@ -60,7 +68,7 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxTopk = 2048;
 constexpr int kNbCompact = 1024; // buckets of the compaction histogram
 
-enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelect = 4 };
+enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelect = 4, kRoleConvert = 5 };
 
 // Optional per-role cycle counters (built only with -DCSA_PROFILE): where each
 // role spends its time, recorded by one thread per role and CTA.
@@ -135,6 +143,7 @@ struct Params {
     int n_chunks;    // d*2 / row_bytes
     // shared memory carve-up (byte offsets from the 1024-aligned base)
     int off_q, off_k, off_w, off_state, off_wg, off_bar, smem_bytes;
+    int off_k8;      // E4M3 keys: staging ring of raw key tiles
     int wg_bytes;    // per-warpgroup scratch
     const uint16_t *q; // only for L2 prefetch; loads go through the tensor map
     const float *w;
@@ -181,8 +190,9 @@ __device__ __forceinline__ Item decode_item(const Params &p, int id)
 }
 
 struct Barriers {
-    uint64_t q_full, q_empty, drain, pad0;
+    uint64_t q_full, q_empty, drain, q_ready;
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
+    uint64_t k8_full[kMaxStages], k8_empty[kMaxStages];  // E4M3 staging ring
     uint64_t acc_full[2], acc_empty[2];
     uint32_t tmem_addr;
     int abort;
@@ -258,17 +268,28 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
         }
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
             const int stage = kload % p.stages;
-            pf.start();
-            if (!wait_bounded(&bars->k_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
-                              kRoleProducer, id))
-                goto unwind;
-            pf.add(pa, kPfProdKEmpty, true);
-            mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
-            uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
             const int row = it.b * p.T + t * kTileKeys;
-            for (int c = 0; c < p.n_chunks; ++c)
-                tma_load_2d(dst + c * kTileKeys * p.row_bytes, tmK, &bars->k_full[stage],
-                            c * (p.row_bytes / 2), row);
+            pf.start();
+            if (p.key_fp8) {
+                // raw E4M3 tile (128 rows x d bytes) into the staging ring
+                if (!wait_bounded(&bars->k8_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
+                                  kRoleProducer, id))
+                    goto unwind;
+                pf.add(pa, kPfProdKEmpty, true);
+                mbar_arrive_expect_tx(&bars->k8_full[stage], static_cast<uint32_t>(kTileKeys * p.d));
+                tma_load_2d(smem + p.off_k8 + stage * kTileKeys * p.d, tmK, &bars->k8_full[stage],
+                            0, row);
+            } else {
+                if (!wait_bounded(&bars->k_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
+                                  kRoleProducer, id))
+                    goto unwind;
+                pf.add(pa, kPfProdKEmpty, true);
+                mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
+                uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
+                for (int c = 0; c < p.n_chunks; ++c)
+                    tma_load_2d(dst + c * kTileKeys * p.row_bytes, tmK, &bars->k_full[stage],
+                                c * (p.row_bytes / 2), row);
+            }
             ++kload;
         }
     }
@@ -277,7 +298,7 @@ unwind:
     for (int s = 0; s < p.stages; ++s) {
         if (kload > s) {
             const int fills = (kload - s + p.stages - 1) / p.stages;
-            wait_drain(&bars->k_full[s], (fills - 1) & 1);
+            wait_drain(p.key_fp8 ? &bars->k8_full[s] : &bars->k_full[s], (fills - 1) & 1);
         }
     }
     if (qload > 0)
@@ -293,14 +314,14 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
     ProfAcc pa;
     Prof pf, pt;
     pt.start();
-    const uint32_t idesc = instr_desc_f16(p.N, 1);
+    const uint32_t idesc = instr_desc_f16(p.N, p.key_fp8 ? 0 : 1); // f16 x f16 for E4M3 keys
     const int ksteps_per_chunk = p.row_bytes / 32;  // 16 elements (32 B) per MMA K step
     const uint32_t q_base = smem_u32(smem + p.off_q);
     const uint32_t k_base = smem_u32(smem + p.off_k);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         pf.start();
-        if (!wait_bounded(&bars->q_full, quse & 1, ctl, kRoleMma, id))
+        if (!wait_bounded(p.key_fp8 ? &bars->q_ready : &bars->q_full, quse & 1, ctl, kRoleMma, id))
             goto unwind;
         pf.add(pa, kPfMmaQFull, true);
         tc_fence_after();
@@ -343,6 +364,101 @@ unwind:
     mma_commit(&bars->drain);
     wait_drain(&bars->drain, 0);
     pa.flush(true);
+}
+
+// ------------------------------------------------------------------ E4M3 converters
+// Byte offset of 16-byte unit `unit` of row r inside one swizzled operand
+// chunk (rows of row_bytes = 128 -> 128-byte swizzle, 64 -> 64-byte swizzle):
+// the unit index is XORed with row bits, as the TMA swizzle modes lay it out.
+__device__ __forceinline__ uint32_t swizzled_unit(int r, int unit, int row_bytes)
+{
+    const uint32_t o = static_cast<uint32_t>(r * row_bytes + unit * 16);
+    const uint32_t mask = row_bytes == 128 ? (7u << 7) : (3u << 7);
+    return o ^ ((o & mask) >> 3);
+}
+
+// Two warps (64 threads, `ct` = 0..63).  Per item: the query block, once the
+// TMA has landed it, from bf16 to f16 in place.  Per key tile: the staged
+// E4M3 tile to f16 in the swizzled key ring.  Each hand-off fences the
+// generic-proxy writes for the tensor cores, then one arrive per warp.
+__device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl,
+                              int ct)
+{
+    const int lane = ct & 31;
+    int kuse = 0, quse = 0;
+    const int units_q = p.N * p.d / 8;                 // 16-byte units of the query block
+    const int units_per_row = p.d / 16;                // 16 E4M3 keys' values per unit
+    const int elems_per_chunk_row = p.row_bytes / 2;
+    for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
+        const Item it = decode_item(p, id);
+        bool ok = wait_bounded(&bars->q_full, quse & 1, ctl, kRoleConvert, id);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok)
+            return;
+        if (it.tile_end > it.tile_begin) {
+            uint4 *qv = reinterpret_cast<uint4 *>(smem + p.off_q);
+            for (int u = ct; u < units_q; u += 64) {
+                uint4 x = qv[u];
+                uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float lo = __uint_as_float(w[i] << 16);
+                    const float hi = __uint_as_float(w[i] & 0xFFFF0000u);
+                    const __half2 h = __floats2half2_rn(lo, hi);
+                    w[i] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                qv[u] = x;
+            }
+            fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&bars->q_ready);
+        ++quse;
+        for (int t = it.tile_begin; t < it.tile_end; ++t) {
+            const int stage = kuse % p.stages;
+            const uint32_t par = (kuse / p.stages) & 1;
+            ok = wait_bounded(&bars->k8_full[stage], par, ctl, kRoleConvert, id);
+            ok = ok && wait_bounded(&bars->k_empty[stage], par ^ 1, ctl, kRoleConvert, id);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                return;
+            const uint4 *src = reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage * kTileKeys * p.d);
+            uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
+            for (int u = ct; u < kTileKeys * units_per_row; u += 64) {
+                const int r = u / units_per_row;
+                const int j0 = (u % units_per_row) * 16;       // first of the unit's 16 values
+                const uint4 x = src[u];
+                const uint32_t *b = reinterpret_cast<const uint32_t *>(&x);
+                uint32_t h[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(
+                        static_cast<__nv_fp8x2_storage_t>(b[i] & 0xFFFFu), __NV_E4M3);
+                    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(
+                        static_cast<__nv_fp8x2_storage_t>(b[i] >> 16), __NV_E4M3);
+                    h[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
+                    h[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int j = j0 + 8 * half;               // 8 values = one 16-byte unit
+                    const int c = j / elems_per_chunk_row;
+                    const int unit = (j % elems_per_chunk_row) / 8;
+                    uint4 *d = reinterpret_cast<uint4 *>(dst + c * kTileKeys * p.row_bytes +
+                                                         swizzled_unit(r, unit, p.row_bytes));
+                    *d = make_uint4(h[4 * half], h[4 * half + 1], h[4 * half + 2], h[4 * half + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->k_full[stage]);
+                mbar_arrive(&bars->k8_empty[stage]);
+            }
+            ++kuse;
+        }
+    }
 }
 
 // ------------------------------------------------------------------ group scratch
@@ -930,9 +1046,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->q_ready, 2);
         for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_full[s], p.key_fp8 ? 2 : 1); // converters, or the TMA's tx
             mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->k8_full[s], 1);
+            mbar_init(&bars->k8_empty[s], 2);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->acc_full[s], 1);
@@ -964,6 +1083,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             run_producer(p, &tmQ, &tmK, smem, bars, ctl);
         else if (warp == 9 && lane == 0)
             run_mma(p, smem, bars, tmem_base, ctl);
+        else if (warp >= 10 && p.key_fp8)
+            run_converter(p, smem, bars, ctl, threadIdx.x - 320);
     }
 
     tc_fence_before();

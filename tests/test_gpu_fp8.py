@@ -1,0 +1,118 @@
+"""E4M3 keys with per-key fp32 scales: CUDA path vs the CPU oracle (needs a B200).
+
+The oracle reads the exact dequantised keys (scale * E4M3 value).  Integer
+inputs use power-of-two scales, so every product and sum is exact in fp32
+and the GPU must match bit for bit; random-normal inputs are judged by recall
+and a 3e-2 relative score tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import check_random_row
+from test_gpu_parity import exact_case, lib, random_case, run_gpu, run_oracle, sample_rows  # noqa: F401
+
+pytestmark = pytest.mark.gpu
+
+
+def fp8(wl):
+    return wl.replace(key_fp8=True)
+
+
+@pytest.mark.parametrize("H", [4, 16, 32, 64, 128])
+def test_fp8_heads_bit_exact(lib, H):
+    wl = workloads.Workload("f8h", B=2, S=300, T=700, H=H, d=128, m=2, topk=100, seed=1200 + H)
+    exact_case(lib, fp8(wl))
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("m", [1, 4])
+def test_fp8_dims_bit_exact(lib, d, m):
+    wl = workloads.Workload("f8d", B=1, S=520, T=900, H=64, d=d, m=m, topk=160, seed=1300 + d + m)
+    exact_case(lib, fp8(wl))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_gate_and_causal_bit_exact(lib, mode, causal):
+    wl = workloads.Workload("f8g", B=1, S=400, T=1500, H=64, d=128, m=4, topk=200, causal=causal,
+                            seed=1400 + mode + 2 * causal)
+    exact_case(lib, fp8(wl), mode=mode)
+
+
+def test_fp8_decode_splits_bit_exact(lib):
+    """Few queries per sequence against many keys: key-range splits, then the
+    select merges the splits' lists."""
+    wl = workloads.Workload("f8s", B=3, S=2, T=20000, H=64, d=128, m=4, topk=512, seed=1500)
+    exact_case(lib, fp8(wl))
+
+
+def test_fp8_scales_and_subnormals(lib):
+    """Keys drawn from every finite E4M3 code (subnormals, zeros of both signs,
+    the largest value) with scales spanning many binades: the GPU must decode
+    every code and apply every scale as the oracle does.  The sums need more
+    than fp32's 24 bits here, so scores are held to 1e-5 relative."""
+    wl = fp8(workloads.Workload("f8c", B=1, S=130, T=256, H=32, d=128, m=1, topk=64,
+                                values="integer", seed=1600))
+    inp = workloads.make_inputs(wl)
+    codes = torch.arange(256, dtype=torch.int32)
+    finite = codes[(codes & 0x7F) != 0x7F].to(torch.uint8)          # drop the NaN codes
+    g = torch.Generator().manual_seed(1601)
+    inp["k"] = finite[torch.randint(0, finite.numel(), (1, wl.T, wl.d), generator=g)].contiguous()
+    inp["k_scale"] = torch.pow(2.0, torch.randint(-8, 6, (1, wl.T), generator=g).float())
+    gi, gs = run_gpu(lib, inp, wl)
+    rows = np.arange(wl.S, dtype=np.int64)
+    check_rows(inp, wl, gi, gs, rows, rtol=1e-5)
+
+
+def check_rows(inp, wl, gi, gs, rows, *, mode=0, rtol):
+    q, w, k, ks = workloads.as_numpy_bits(inp)
+    ri, _, _, rc = oracle.topk(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
+                               topk=wl.topk, causal=wl.causal, mode=mode, rows=rows)
+    gi = gi.reshape(-1, wl.topk)
+    gs = gs.reshape(-1, wl.topk)
+    for n, row in enumerate(rows):
+        b, i = divmod(int(row), wl.S)
+        I, vis = oracle.score_row(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
+                                  b=b, i=i, causal=wl.causal)
+        check_random_row(gi[row], gs[row], ri[n], rc[n], I, vis, topk=wl.topk, gate=mode == 1,
+                         rtol=rtol, label=f"{wl.name} row {row}")
+
+
+def test_fp8_random_recall(lib):
+    wl = workloads.Workload("f8r", B=2, S=900, T=1200, H=64, d=128, m=1, topk=256, seed=1700)
+    random_case(lib, fp8(wl), sample_rows(wl, 40), rtol=3e-2)
+
+
+def test_fp8_random_gate(lib):
+    wl = workloads.Workload("f8q", B=1, S=700, T=2400, H=64, d=128, m=2, topk=300, seed=1701)
+    random_case(lib, fp8(wl), sample_rows(wl, 30), mode=1, rtol=3e-2)
+
+
+@pytest.mark.slow
+def test_long_prefill_fp8_full_size(lib):
+    """Long prefill (S=262,144, T=65,536, E4M3 keys) at full size, sampled queries."""
+    wl = workloads.CONFIGS["long_prefill_fp8"]
+    random_case(lib, wl, sample_rows(wl, 6, seed=3), rtol=3e-2)
+
+
+@pytest.mark.slow
+def test_long_prefill_fp8_gated_full_size(lib):
+    wl = workloads.CONFIGS["long_prefill_fp8_gated"]
+    random_case(lib, wl, sample_rows(wl, 6, seed=4), mode=1, rtol=3e-2)
+
+
+@pytest.mark.slow
+def test_decode_fp8_full_size(lib):
+    """Batched decode (B=32 x 64 queries at T=131,072, E4M3 keys), sampled queries."""
+    wl = workloads.CONFIGS["decode_fp8"]
+    random_case(lib, wl, sample_rows(wl, 8, seed=5), rtol=3e-2)
+
+
+@pytest.mark.slow
+def test_decode1_fp8_full_size(lib):
+    """One query per sequence (B=32, T=131,072, E4M3 keys), sampled queries."""
+    wl = workloads.CONFIGS["decode1_fp8"]
+    random_case(lib, wl, sample_rows(wl, 4, seed=6), rtol=3e-2)

@@ -18,7 +18,9 @@ context).  Value distributions:
   w ~ N(0, 1/H_I) in fp32;
 * FP8 keys: k ~ N(0, 1) in fp32, per-key scale = max_j |k[s, j]| / 448,
   bytes = E4M3(k / scale) with round-to-nearest-even (torch's
-  ``float8_e4m3fn`` cast).  The effective key is scale * E4M3 value.
+  ``float8_e4m3fn`` cast).  The effective key is scale * E4M3 value.  With
+  integer values the bytes encode 4*k (integers in [-4, 4], exact in E4M3)
+  and every scale is 1/4, so the effective keys equal the integer recipe's.
 """
 from __future__ import annotations
 
@@ -162,7 +164,11 @@ def make_inputs(wl: Workload, device="cpu", seed: Optional[int] = None, chunk_ro
         k32 = _integer_quarters((B, T, d), g, device)
     else:
         k32 = torch.randn((B, T, d), generator=g, device=device)
-    if wl.key_fp8:
+    if wl.key_fp8 and wl.values == "integer":
+        # 4*k is an integer in [-4, 4]: exact in E4M3, scale 1/4 exact in fp32
+        k = (k32 * 4.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        k_scale = torch.full((B, T), 0.25, dtype=torch.float32, device=device)
+    elif wl.key_fp8:
         k, k_scale = quantize_e4m3(k32)
     else:
         k, k_scale = k32.to(torch.bfloat16), None
