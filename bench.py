@@ -385,13 +385,24 @@ def main():
     fused_avg = statistics.mean(fused_ms)
     k_tflops = flops / (fused_avg / 1000.0) / 1e12
     sha = kernel_sources_sha()
-    roofline = {"bound": "tensor", "achieved": k_tflops, "peak": peak, "unit": "TFLOP/s",
-                "frac": k_tflops / peak if peak else None,
-                "traffic": measured_traffic(wl.name, sha),
-                "peak_source": f"{peak_src} bf16 dense ({'sustained' if sustained else 'burst'})",
-                "kernel": "indexer_topk_kernel (fused scoring + candidate filter)",
-                "kernel_ms": fused_avg, "select_kernel_ms": statistics.mean(select_ms),
-                "algorithmic_flops_per_launch": flops, "sources_sha": sha}
+    alg_bytes = wl.input_bytes() + wl.output_bytes()
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    common = {"traffic": measured_traffic(wl.name, sha),
+              "kernel": "indexer_topk_kernel (fused scoring + candidate filter)",
+              "kernel_ms": fused_avg, "select_kernel_ms": statistics.mean(select_ms),
+              "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
+              "sources_sha": sha}
+    if flops / alg_bytes < ridge:
+        # few queries per key (single-query decode): the key stream bounds it
+        gbs = alg_bytes / (fused_avg / 1000.0) / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth",
+                    **common}
+    else:
+        roofline = {"bound": "tensor", "achieved": k_tflops, "peak": peak, "unit": "TFLOP/s",
+                    "frac": k_tflops / peak if peak else None,
+                    "peak_source": f"{peak_src} bf16 dense ({'sustained' if sustained else 'burst'})",
+                    **common}
     cpu = None
     if not args.no_cpu_baseline:
         cpu_inputs = inputs_for_oracle(wl, {"q": q, "w": w, "k": k, "k_scale": ks})
@@ -401,7 +412,8 @@ def main():
     line = {
         "metric": "indexer queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 x e4m3 (f16 MMA)" if wl.key_fp8 else "bf16",
         "data": "synthetic", "config": config_dict(wl), "tflops": tflops,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * plan.launches,

@@ -377,18 +377,64 @@ __device__ __forceinline__ uint32_t swizzled_unit(int r, int unit, int row_bytes
     return o ^ ((o & mask) >> 3);
 }
 
+// Four E4M3 values (one 32-bit word) -> four f16 (two words), exact.
+__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t b)
+{
+    uint2 r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}\n"
+        : "=r"(r.x), "=r"(r.y)
+        : "r"(b));
+    return r;
+}
+
+// Two bf16 (one word) -> two f16 (one word), round to nearest.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+        : "=r"(r)
+        : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(__uint_as_float(w << 16)));
+    return r;
+}
+
+constexpr int kConvThreads = 64;
+constexpr int kConvUnits = kTileKeys * 128 / 16 / kConvThreads; // 16-value units per thread (d <= 128)
+
 // Two warps (64 threads, `ct` = 0..63).  Per item: the query block, once the
 // TMA has landed it, from bf16 to f16 in place.  Per key tile: the staged
-// E4M3 tile to f16 in the swizzled key ring.  Each hand-off fences the
-// generic-proxy writes for the tensor cores, then one arrive per warp.
+// E4M3 tile to f16 in the swizzled key ring; a thread's units (and so its
+// source and destination offsets) are the same for every tile.  Each hand-off
+// fences the generic-proxy writes for the tensor cores, then one arrive per
+// warp.
 __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl,
                               int ct)
 {
     const int lane = ct & 31;
     int kuse = 0, quse = 0;
     const int units_q = p.N * p.d / 8;                 // 16-byte units of the query block
-    const int units_per_row = p.d / 16;                // 16 E4M3 keys' values per unit
+    const int units_per_row = p.d / 16;                // 16 E4M3 values per unit
+    const int n_units = kTileKeys * units_per_row / kConvThreads;
     const int elems_per_chunk_row = p.row_bytes / 2;
+    // Unit i of this thread is u = 64 i + ct: row 64 i / units_per_row + ct /
+    // units_per_row (a multiple of 8 rows apart for d <= 128, so the swizzle
+    // term is the same for every i) and the same columns for every i.
+    uint32_t dst_base[2];
+    {
+        const int r0 = ct / units_per_row;
+        const int j0 = (ct % units_per_row) * 16;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int j = j0 + 8 * half;
+            const int c = j / elems_per_chunk_row;
+            const int unit = (j % elems_per_chunk_row) / 8;
+            dst_base[half] =
+                static_cast<uint32_t>(c * kTileKeys * p.row_bytes) + swizzled_unit(r0, unit, p.row_bytes);
+        }
+    }
+    const uint32_t dst_step = static_cast<uint32_t>(kConvThreads / units_per_row * p.row_bytes);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         bool ok = wait_bounded(&bars->q_full, quse & 1, ctl, kRoleConvert, id);
@@ -397,16 +443,12 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
             return;
         if (it.tile_end > it.tile_begin) {
             uint4 *qv = reinterpret_cast<uint4 *>(smem + p.off_q);
-            for (int u = ct; u < units_q; u += 64) {
+            for (int u = ct; u < units_q; u += kConvThreads) {
                 uint4 x = qv[u];
-                uint32_t *w = reinterpret_cast<uint32_t *>(&x);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float lo = __uint_as_float(w[i] << 16);
-                    const float hi = __uint_as_float(w[i] & 0xFFFF0000u);
-                    const __half2 h = __floats2half2_rn(lo, hi);
-                    w[i] = *reinterpret_cast<const uint32_t *>(&h);
-                }
+                x.x = bf16x2_to_f16x2(x.x);
+                x.y = bf16x2_to_f16x2(x.y);
+                x.z = bf16x2_to_f16x2(x.z);
+                x.w = bf16x2_to_f16x2(x.w);
                 qv[u] = x;
             }
             fence_proxy_async_smem();
@@ -423,31 +465,19 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 return;
-            const uint4 *src = reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage * kTileKeys * p.d);
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage * kTileKeys * p.d);
             uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
-            for (int u = ct; u < kTileKeys * units_per_row; u += 64) {
-                const int r = u / units_per_row;
-                const int j0 = (u % units_per_row) * 16;       // first of the unit's 16 values
-                const uint4 x = src[u];
-                const uint32_t *b = reinterpret_cast<const uint32_t *>(&x);
-                uint32_t h[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(
-                        static_cast<__nv_fp8x2_storage_t>(b[i] & 0xFFFFu), __NV_E4M3);
-                    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(
-                        static_cast<__nv_fp8x2_storage_t>(b[i] >> 16), __NV_E4M3);
-                    h[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
-                    h[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
-                }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int j = j0 + 8 * half;               // 8 values = one 16-byte unit
-                    const int c = j / elems_per_chunk_row;
-                    const int unit = (j % elems_per_chunk_row) / 8;
-                    uint4 *d = reinterpret_cast<uint4 *>(dst + c * kTileKeys * p.row_bytes +
-                                                         swizzled_unit(r, unit, p.row_bytes));
-                    *d = make_uint4(h[4 * half], h[4 * half + 1], h[4 * half + 2], h[4 * half + 3]);
+            for (int i = 0; i < kConvUnits; ++i) {
+                if (i < n_units) {
+                    const uint4 x = src[i * kConvThreads + ct];
+                    const uint2 a = e4m3x4_to_f16x4(x.x);
+                    const uint2 b = e4m3x4_to_f16x4(x.y);
+                    const uint2 c = e4m3x4_to_f16x4(x.z);
+                    const uint2 d = e4m3x4_to_f16x4(x.w);
+                    *reinterpret_cast<uint4 *>(dst + dst_base[0] + i * dst_step) = make_uint4(a.x, a.y, b.x, b.y);
+                    *reinterpret_cast<uint4 *>(dst + dst_base[1] + i * dst_step) = make_uint4(c.x, c.y, d.x, d.y);
                 }
             }
             fence_proxy_async_smem();
