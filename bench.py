@@ -224,11 +224,22 @@ def main():
                     help="query rows the oracle computes per reference step")
     ap.add_argument("--cpu-rows", type=int, default=512,
                     help="query rows of the CPU-baseline sample (rank 0)")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a workload field (B, S, T, H, d, m, topk, seed, key_fp8, "
+                         "gated), e.g. for a reduced profiling shape; the workload name records it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = workloads.CONFIGS[args.config]
+    if args.set:
+        kw = {}
+        for item in args.set:
+            field, _, value = item.partition("=")
+            if field not in ("B", "S", "T", "H", "d", "m", "topk", "seed", "key_fp8", "gated"):
+                raise SystemExit(f"--set: unknown field {field!r}")
+            kw[field] = (value.lower() in ("1", "true")) if field in ("key_fp8", "gated") else int(value)
+        wl = wl.replace(name=wl.name + "[" + ",".join(args.set) + "]", **kw)
 
     if args.impl == "reference":
         return run_reference(args, wl)
