@@ -82,7 +82,7 @@ struct Plan {
     int qb_chunk;      // query blocks per batch in one launch chunk
     int chunks;
     int fast_fc, fast_fq; // epilogue fast path (0 = generic)
-    size_t ws_lists, ws_counts, ws_total;
+    size_t ws_lists, ws_counts, ws_scores, ws_total;
 };
 
 csa_status_t validate(const csa_args_t *a)
@@ -180,13 +180,12 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     p.n_wg = (qps >= 2 && p.N >= 64) ? 2 : 1;
     p.qpw = qps / p.n_wg;
 
-    p.cap = 2 * p.topk;
-    if (p.cap < p.topk + 256)
-        p.cap = p.topk + 256;
-    p.cap = (p.cap + 127) / 128 * 128;
-    if (p.cap > csa::kGroupThreads * csa::kEpt)
-        return CSA_ERR_UNSUPPORTED;
-    p.slack = (p.cap - csa::kTileKeys - p.topk) / 2;
+    // Candidate list per (query, split): the top k plus room for the
+    // selector's histogram bucket around the k-th score.
+    int extra = p.topk / 4;
+    if (extra < 256)
+        extra = 256;
+    p.cap = (p.topk + extra + 127) / 128 * 128;
 
     // per pipeline stage: the MMA's 16-bit key tile, plus (E4M3 keys) the raw
     // staged tile it is converted from
@@ -196,11 +195,9 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     off += p.N * p.d * 2;
     p.off_k = off;
     int tail = 0;
-    tail += p.qps * p.H * 4;                                   // w
+    tail += 2 * p.qps * p.H * 4;                               // w, one half per item parity
     tail = (tail + 15) / 16 * 16;
-    tail += p.qps * static_cast<int>(sizeof(csa::QueryState));
-    p.wg_bytes = (static_cast<int>(sizeof(csa::WgScratch)) + 15) / 16 * 16;
-    tail += 2 * p.wg_bytes;
+    tail += (static_cast<int>(sizeof(csa::SelectorScratch)) + 15) / 16 * 16;
     tail += static_cast<int>(sizeof(csa::Barriers)) + 16;
     int stages = (kSmemLimit - 1024 - off - tail) / k_stage;
     if (stages > csa::kMaxStages)
@@ -213,13 +210,10 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     if (p.key_fp8)
         off += stages * csa::kTileKeys * p.d;
     p.off_w = off;
-    off += p.qps * p.H * 4;
+    off += 2 * p.qps * p.H * 4;
     off = (off + 15) / 16 * 16;
-    p.off_state = off;
-    off += p.qps * static_cast<int>(sizeof(csa::QueryState));
-    off = (off + 15) / 16 * 16;
-    p.off_wg = off;
-    off += 2 * p.wg_bytes;
+    p.off_sel = off;
+    off += (static_cast<int>(sizeof(csa::SelectorScratch)) + 15) / 16 * 16;
     p.off_bar = off;
     off += static_cast<int>(sizeof(csa::Barriers));
     p.smem_bytes = off + 1024;
@@ -252,21 +246,39 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
             }
         }
     }
+    const int tiles_max = max_tiles(a, p.q_offset);
+    const int min_split = (tiles_max * csa::kTileKeys + csa::kMaxItemKeys - 1) / csa::kMaxItemKeys;
+    if (nsplit < min_split)
+        nsplit = min_split;
     if (nsplit < 1 || nsplit > csa::kSelMaxSplits)
         return CSA_ERR_UNSUPPORTED;
     p.nsplit = nsplit;
+    // keys of the longest item: its split's share of the heaviest query block's tiles
+    p.nmax = (tiles_max + nsplit - 1) / nsplit * csa::kTileKeys;
+    if (p.nmax < csa::kTileKeys)
+        p.nmax = csa::kTileKeys;
 
+    // Score buffers: per CTA two halves of qps x nmax fp32 (grid-sized, not
+    // S-sized).  A budget that cannot hold a full grid's buffers next to one
+    // query block's lists runs fewer CTAs.
+    int grid = sms;
+    const size_t scores_per_cta = static_cast<size_t>(2) * p.qps * p.nmax * 4;
     // Candidate lists: one per (query, split), cap keys each, plus its length.
     // A launch chunk covers qb_chunk query blocks of every batch.
     const size_t rows_per_qb = static_cast<size_t>(p.B) * p.qps;
     const size_t lists_per_qb = rows_per_qb * nsplit * p.cap * 8;
     const size_t counts_per_qb = rows_per_qb * nsplit * 4;
     const size_t per_qb = lists_per_qb + counts_per_qb;
+    if (static_cast<size_t>(grid) * scores_per_cta + per_qb + 1024 > ws_cap) {
+        if (ws_cap < per_qb + scores_per_cta + 1024)
+            return CSA_ERR_WORKSPACE;
+        const size_t fit = (ws_cap - per_qb - 1024) / scores_per_cta;
+        grid = static_cast<int>(fit < static_cast<size_t>(grid) ? fit : grid);
+    }
+    const size_t ws_scores = align256(static_cast<size_t>(grid) * scores_per_cta);
     long long qb_chunk = nqb_total;
-    if (ws_cap < 512 + per_qb)
-        return CSA_ERR_WORKSPACE;
-    if (static_cast<size_t>(qb_chunk) * per_qb + 512 > ws_cap)
-        qb_chunk = static_cast<long long>((ws_cap - 512) / per_qb);
+    if (static_cast<size_t>(qb_chunk) * per_qb + ws_scores + 1024 > ws_cap)
+        qb_chunk = static_cast<long long>((ws_cap - ws_scores - 1024) / per_qb);
     if (qb_chunk < 1)
         return CSA_ERR_WORKSPACE;
     const long long items = static_cast<long long>(p.B) * qb_chunk * nsplit;
@@ -280,12 +292,13 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     plan.nqb_total = nqb_total;
     plan.qb_chunk = static_cast<int>(qb_chunk);
     plan.chunks = static_cast<int>((nqb_total + qb_chunk - 1) / qb_chunk);
-    plan.grid = p.n_items < sms ? p.n_items : sms;
+    plan.grid = p.n_items < grid ? p.n_items : grid;
     if (plan.grid < 1)
         plan.grid = 1;
     plan.ws_lists = align256(static_cast<size_t>(qb_chunk) * lists_per_qb);
     plan.ws_counts = align256(static_cast<size_t>(qb_chunk) * counts_per_qb);
-    plan.ws_total = plan.ws_lists + plan.ws_counts;
+    plan.ws_scores = ws_scores;
+    plan.ws_total = plan.ws_lists + plan.ws_counts + plan.ws_scores;
     // Epilogue fast path: whole 32-column queries, 64 or 128 columns per group.
     const int cols = p.qpw * p.H;
     plan.fast_fc = (p.H >= 32 && (cols == 64 || cols == 128)) ? cols : 0;
@@ -343,6 +356,7 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
     p.k_scale = a->k_scale;
     p.lists = reinterpret_cast<uint64_t *>(ws);
     p.counts = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + plan.ws_lists);
+    p.scores = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + plan.ws_lists + plan.ws_counts);
     p.wait_limit = static_cast<long long>(g_wait_limit);
 
     CUtensorMap tmQ, tmK;

@@ -1,5 +1,5 @@
-// indexer_kernel.cuh -- the fused lightning-indexer scoring + streaming
-// candidate filter.
+// indexer_kernel.cuh -- the fused lightning-indexer scoring + candidate
+// selection kernel.
 //
 // One persistent CTA per SM walks work items (batch b, block of qps queries,
 // range of key tiles).  For each 128-key tile the tensor cores compute the
@@ -8,32 +8,34 @@
 // Top-k", abstract: the lightning indexer scores compressed keys per query),
 // with keys as the MMA's M dimension so that each TMEM lane holds one key's
 // logits for every (query, head).  The epilogue applies ReLU and the head
-// weights, masks keys the query may not see, and streams the surviving
-// (score, index) pairs into the query's candidate list in global memory; a
-// list that could overflow is cut back in place to the top k plus slack and
-// the admission bound rises to the smallest score kept.  When an item's key
-// range is done the list holds a superset of the query's top k over that
-// range; select_kernel.cuh turns the lists into the exact, sorted top k.  The
-// [B,S,H_I,T] score tensor never exists and the extra memory is O(S * k).
+// weights and writes one fp32 score per (query, key) into the CTA's score
+// buffer for the item (two halves, alternating between items).  A selector
+// warpgroup then cuts each query's scores of a finished item down to a
+// candidate list of at most `cap` keys that holds the query's top k over the
+// item's key range (exactly the top k when a cut is needed), while the
+// epilogue already fills the other half.  select_kernel.cuh turns the lists
+// into the exact, sorted top k.  No score tensor over all queries exists: the
+// buffers are per CTA (grid x 2 x qps x keys per item) and the lists O(S*k).
 //
-// Warp roles (384 threads, three warpgroups):
-//   warps 0..3  epilogue warpgroup 0: the first half of the item's queries
-//   warps 4..7  epilogue warpgroup 1: the second half (idle when qps == 1)
-//   warp 8      TMA producer: the query block once per item (with an L2
-//               prefetch of the next item's), key tiles into a ring
-//   warp 9      TMEM owner and MMA issuer (one thread): per key tile, d/16
-//               tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
-//               256-column TMEM accumulators
-//   warps 10,11 E4M3 keys only: converters.  The producer lands each FP8 key
-//               tile in a staging ring; the converters rewrite it as f16
-//               into the MMA's swizzled key ring (exact: every E4M3 value is
-//               an f16 normal) and convert the item's query block from bf16
-//               to f16 in place (exact for |q| < 65504), so the MMA runs
-//               kind::f16 with both operands f16.  The key's fp32 scale
-//               multiplies its score after the head reduction (scale > 0).
-// The block launches with 168 registers per thread; the producer/MMA
-// warpgroup gives most of its share to the two epilogue warpgroups
-// (3 x 128 x 168 = 2 x 128 x kEpiRegs + 128 x kCtlRegs).
+// Warp roles (512 threads, four warpgroups):
+//   warps 0..3   epilogue warpgroup 0: the first half of the item's queries
+//   warps 4..7   epilogue warpgroup 1: the second half (idle when qps == 1)
+//   warp 8       TMA producer: the query block once per item (with an L2
+//                prefetch of the next item's), key tiles into a ring
+//   warp 9       TMEM owner and MMA issuer (one thread): per key tile, d/16
+//                tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
+//                256-column TMEM accumulators
+//   warps 10,11  E4M3 keys only: converters.  The producer lands each FP8 key
+//                tile in a staging ring; the converters rewrite it as f16
+//                into the MMA's swizzled key ring (exact: every E4M3 value is
+//                an f16 normal) and convert the item's query block from bf16
+//                to f16 in place (exact for |q| < 65504), so the MMA runs
+//                kind::f16 with both operands f16.  The key's fp32 scale
+//                multiplies its score after the head reduction (scale > 0).
+//   warps 12..15 selector
+// The block launches with 128 registers per thread; the two control
+// warpgroups give most of their share to the epilogue warpgroups
+// (4 x 128 x 128 = 2 x 128 x kEpiRegs + 2 x 128 x kCtlRegs).
 //
 // Epilogue fast path (H_I >= 32, at most 128 TMEM columns per warpgroup): a
 // warp reads its 32 TMEM lanes with two 16-lane x 256-bit loads, so every
@@ -55,18 +57,18 @@ namespace csa {
 
 constexpr int kTileKeys = 128;   // MMA M: keys per tile
 constexpr int kSlotCols = 256;   // TMEM columns per accumulator slot
-constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;  // registers per thread the kernel must be built with
-constexpr int kEpiRegs = 216;     // after the split: epilogue warpgroups
-constexpr int kCtlRegs = 72;      //                  producer / MMA warpgroup
-static_assert(2 * 128 * kEpiRegs + 128 * kCtlRegs == kThreads * kLaunchRegs,
+constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 128;  // registers per thread the kernel must be built with
+constexpr int kEpiRegs = 160;     // after the split: epilogue warpgroups
+constexpr int kCtlRegs = 96;      //                  producer / MMA / converters, selector
+static_assert(2 * 128 * kEpiRegs + 2 * 128 * kCtlRegs == kThreads * kLaunchRegs,
               "register split must match the launch budget");
 constexpr int kGroupThreads = 128;
-constexpr int kBarWg0 = 1, kBarWg1 = 2;  // named barriers of the epilogue warpgroups
-constexpr int kEpt = 32;         // candidate keys per thread in a group (cap <= 4096)
+constexpr int kBarWg0 = 1, kBarWg1 = 2, kBarSelect = 3;  // named barriers
 constexpr int kMaxStages = 8;
 constexpr int kMaxTopk = 2048;
-constexpr int kNbCompact = 1024; // buckets of the compaction histogram
+constexpr int kNbSelect = 2048;  // buckets of the selector's histogram
+constexpr int kMaxItemKeys = 65536; // keys of one work item (longer ranges are split)
 
 enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelect = 4, kRoleConvert = 5 };
 
@@ -74,8 +76,8 @@ enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelec
 // role spends its time, recorded by one thread per role and CTA.
 enum ProfSlot : int {
     kPfProdQEmpty, kPfProdKEmpty, kPfMmaQFull, kPfMmaKFull, kPfMmaAccEmpty, kPfMmaTotal,
-    kPfEpiAccFull, kPfEpiCompact, kPfEpiTotal, kPfEpiCompactCount, kPfEpiTiles, kPfEpiMath,
-    kPfEpiTileBar, kPfSlots
+    kPfEpiAccFull, kPfEpiBufEmpty, kPfEpiTotal, kPfEpiTiles, kPfEpiMath, kPfSelBufFull,
+    kPfSelBusy, kPfSelTotal, kPfSelCut, kPfSlots
 };
 #ifdef CSA_PROFILE
 constexpr int kProfCtas = 160;
@@ -138,18 +140,18 @@ struct Params {
     int n_items;
     int stages;
     int cap;      // candidate list capacity per query and split
-    int slack;    // compaction keeps at most topk + slack when it must cut exactly
+    int nmax;     // score-buffer keys per query (the longest item's key range)
     int row_bytes;   // bytes of one swizzled operand row: min(128, 2*d)
     int n_chunks;    // d*2 / row_bytes
     // shared memory carve-up (byte offsets from the 1024-aligned base)
-    int off_q, off_k, off_w, off_state, off_wg, off_bar, smem_bytes;
+    int off_q, off_k, off_w, off_sel, off_bar, smem_bytes;
     int off_k8;      // E4M3 keys: staging ring of raw key tiles
-    int wg_bytes;    // per-warpgroup scratch
     const uint16_t *q; // only for L2 prefetch; loads go through the tensor map
     const float *w;
     const float *k_scale;
     uint64_t *lists; // [list row][nsplit][cap] candidate keys
     int *counts;     // [list row][nsplit] keys in each list
+    float *scores;   // [gridDim.x][2][qps][nmax] the item's scores
     long long wait_limit;
 };
 
@@ -194,16 +196,9 @@ struct Barriers {
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t k8_full[kMaxStages], k8_empty[kMaxStages];  // E4M3 staging ring
     uint64_t acc_full[2], acc_empty[2];
+    uint64_t buf_full[2], buf_empty[2];                   // score-buffer halves
     uint32_t tmem_addr;
     int abort;
-};
-
-// Per-query streaming state of the current item.
-struct QueryState {
-    int cnt;          // candidates in the list
-    uint32_t bound;   // admit a key only if ord(score) >= bound
-    int vis_end;      // keys s < vis_end are visible to this query
-    int pad;
 };
 
 // Bounded wait used when unwinding: ignores the abort flag and the (possibly
@@ -491,214 +486,6 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
     }
 }
 
-// ------------------------------------------------------------------ group scratch
-struct WgScratch {          // one per epilogue warpgroup
-    GroupSmall gs;
-    uint32_t hist[kNbCompact];
-};
-
-// ------------------------------------------------------------------ compaction
-// Bucket of the k-th largest key over a 1024-bucket histogram of the group:
-// {b*, keys in buckets above b*, keys in b*} with above < need <= above + in.
-// Thread tid owns buckets [8 tid, 8 tid + 8); two group barriers.
-__device__ __forceinline__ void compact_boundary(const uint32_t *hist, int need, GroupSmall *gs,
-                                                 int bar, int tid, int (&out)[3])
-{
-    constexpr int PER = kNbCompact / kGroupThreads;
-    const int lane = tid & 31, wid = tid >> 5;
-    uint32_t c[PER];
-    uint32_t sum = 0;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-        c[j] = hist[tid * PER + j];
-        sum += c[j];
-    }
-    uint32_t suf = sum; // inclusive suffix sum over the warp's threads
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
-        if (lane + off < 32)
-            suf += t;
-    }
-    if (lane == 0)
-        gs->warp_sums[wid] = suf;
-    named_bar_sync(bar, kGroupThreads);
-    uint32_t higher = 0;
-#pragma unroll
-    for (int w = 0; w < kGroupThreads / 32; ++w)
-        higher += w > wid ? gs->warp_sums[w] : 0u;
-    const uint32_t above_thread = suf - sum + higher;
-    const uint32_t nd = static_cast<uint32_t>(need);
-    if (above_thread < nd && nd <= above_thread + sum) {
-        uint32_t above = above_thread;
-#pragma unroll
-        for (int j = PER - 1; j >= 0; --j) {
-            if (above + c[j] >= nd) {
-                gs->bcast[0] = tid * PER + j;
-                gs->bcast[1] = static_cast<int>(above);
-                gs->bcast[2] = static_cast<int>(c[j]);
-                break;
-            }
-            above += c[j];
-        }
-    }
-    named_bar_sync(bar, kGroupThreads);
-    out[0] = gs->bcast[0];
-    out[1] = gs->bcast[1];
-    out[2] = gs->bcast[2];
-}
-
-// Cuts a query's list back when it could overflow: keeps every key whose
-// bucket is at or above the bucket of the k-th largest key -- a superset of
-// the top k -- or, when that bucket is too full, the radix-exact top k plus
-// slack.  Buckets split the list's own [min, max] range of score order images
-// into 1024 equal integer ranges.  Warp w owns list slots [1024 w, 1024 w +
-// 1024) (lane l: slots 1024 w + 64 i + 2 l and the one after) and writes the
-// keys it keeps back with coalesced stores.  Updates cnt and raises bound to
-// the smallest kept score.  The group's histogram is all zero on entry and on
-// return.
-__device__ void compact_list(const Params &p, uint64_t *list, QueryState &st, WgScratch *sc,
-                             int bar, int tid)
-{
-    const int n = st.cnt;
-    const int lane = tid & 31, wid = tid >> 5;
-    uint64_t e[kEpt];
-#pragma unroll
-    for (int i = 0; i < kEpt / 2; ++i) {
-        const int j = wid * (kEpt * 32) + i * 64 + 2 * lane;
-        if (j + 1 < n) {
-            const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(list + j);
-            e[2 * i] = v.x;
-            e[2 * i + 1] = v.y;
-        } else {
-            e[2 * i] = j < n ? list[j] : 0ull;
-            e[2 * i + 1] = 0ull;
-        }
-    }
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll
-    for (int i = 0; i < kEpt; ++i) {
-        if (e[i] != 0) {
-            lo = min(lo, key_ord(e[i]));
-            hi = max(hi, key_ord(e[i]));
-        }
-    }
-    lo = __reduce_min_sync(0xffffffffu, lo);
-    hi = __reduce_max_sync(0xffffffffu, hi);
-    if (lane == 0) {
-        sc->gs.warp_sums[wid] = lo;
-        sc->gs.warp_sums[16 + wid] = hi;
-    }
-    named_bar_sync(bar, kGroupThreads);
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-    for (int w = 0; w < kGroupThreads / 32; ++w) {
-        mn = min(mn, sc->gs.warp_sums[w]);
-        mx = max(mx, sc->gs.warp_sums[16 + w]);
-    }
-    const uint32_t span = mx - mn;
-    const int shift = span < static_cast<uint32_t>(kNbCompact) ? 0 : 32 - __clz(span) - 10;
-    int bk[kEpt]; // each key's bucket, -1 for an empty slot
-#pragma unroll
-    for (int i = 0; i < kEpt; ++i) {
-        bk[i] = e[i] != 0 ? static_cast<int>((key_ord(e[i]) - mn) >> shift) : -1;
-        if (bk[i] >= 0)
-            atomicAdd(&sc->hist[bk[i]], 1u);
-    }
-    named_bar_sync(bar, kGroupThreads);
-    int bd[3];
-    compact_boundary(sc->hist, p.topk, &sc->gs, bar, tid, bd);
-    // every thread read its own buckets in compact_boundary: clear them
-#pragma unroll
-    for (int j = 0; j < kNbCompact / kGroupThreads; ++j)
-        sc->hist[tid * (kNbCompact / kGroupThreads) + j] = 0;
-    const int bstar = bd[0];
-    const int cand_kept = bd[1] + bd[2];
-    uint32_t newmin = 0xFFFFFFFFu;
-    int kept = 0;
-    if (cand_kept <= p.cap - 2 * kTileKeys) {
-        uint32_t keep = 0;
-        int mine = 0;
-        uint32_t kmin = 0xFFFFFFFFu;
-#pragma unroll
-        for (int i = 0; i < kEpt; ++i) {
-            const bool k = bk[i] >= bstar;
-            keep |= k ? (1u << i) : 0u;
-            mine += k ? 1 : 0;
-            kmin = k ? min(kmin, key_ord(e[i])) : kmin;
-        }
-        const int wcount = __reduce_add_sync(0xffffffffu, mine);
-        kmin = __reduce_min_sync(0xffffffffu, kmin);
-        if (lane == 0) {
-            sc->gs.warp_sums[wid] = static_cast<uint32_t>(wcount);
-            sc->gs.warp_sums[16 + wid] = kmin;
-        }
-        named_bar_sync(bar, kGroupThreads);
-        int pos = 0;
-#pragma unroll
-        for (int w = 0; w < kGroupThreads / 32; ++w) {
-            const int c = static_cast<int>(sc->gs.warp_sums[w]);
-            pos += w < wid ? c : 0;
-            kept += c;
-            newmin = min(newmin, sc->gs.warp_sums[16 + w]);
-        }
-        const unsigned lt = lanemask_lt();
-#pragma unroll
-        for (int i = 0; i < kEpt; ++i) {
-            const bool k = (keep >> i) & 1u;
-            const unsigned m = __ballot_sync(0xffffffffu, k);
-            if (k)
-                list[pos + __popc(m & lt)] = e[i];
-            pos += __popc(m);
-        }
-    } else {
-        int k2;
-        const uint64_t L = radix_bound<kGroupThreads, kEpt>(e, p.topk, p.slack, sc->hist, &sc->gs,
-                                                            bar, tid, &k2);
-        kept = write_kept<kGroupThreads, kEpt>(e, L, list, &sc->gs, bar, tid, &newmin);
-        for (int i = tid; i < kNbCompact; i += kGroupThreads)
-            sc->hist[i] = 0;
-    }
-    named_bar_sync(bar, kGroupThreads); // list writes and scratch reads done
-    if (tid == 0) {
-        st.cnt = kept;
-        st.bound = max(st.bound, newmin);
-    }
-    named_bar_sync(bar, kGroupThreads);
-}
-
-// ------------------------------------------------------------------ emission
-// Appends this warp's surviving (score, key) pairs of Q queries to their
-// candidate lists: one ballot per query, the lane-0 atomics back to back.
-// Query j's list starts at lbase + j * lstride.
-template <int Q>
-__device__ __forceinline__ void emit_batch(const float *sc, int j0, int s, float kscale,
-                                           QueryState *qs, uint64_t *lbase, size_t lstride,
-                                           int lane)
-{
-    uint32_t ord[Q];
-    unsigned bal[Q];
-    int base[Q];
-#pragma unroll
-    for (int q = 0; q < Q; ++q) {
-        const QueryState st = qs[j0 + q];
-        ord[q] = ord_of_score(sc[q] * kscale);
-        bal[q] = __ballot_sync(0xffffffffu, s < st.vis_end && ord[q] >= st.bound);
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int q = 0; q < Q; ++q)
-            base[q] = bal[q] ? atomicAdd(&qs[j0 + q].cnt, __popc(bal[q])) : 0;
-    }
-#pragma unroll
-    for (int q = 0; q < Q; ++q) {
-        base[q] = __shfl_sync(0xffffffffu, base[q], 0);
-        if (bal[q] & (1u << lane))
-            lbase[static_cast<size_t>(j0 + q) * lstride + base[q] +
-                  __popc(bal[q] & lanemask_lt())] = make_key(ord[q], static_cast<uint32_t>(s));
-    }
-}
-
 // ------------------------------------------------------------------ fast tile math
 template <int FC> struct Ld16x256;
 template <> struct Ld16x256<64> {
@@ -798,38 +585,6 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
     }
 }
 
-// Appends this warp's surviving keys of FQ queries (one key per thread, the
-// queries' admission bounds and visibility ends cached in registers).
-template <int FQ>
-__device__ __forceinline__ void fast_emit(const float (&F)[FQ], const uint32_t (&bnd)[FQ],
-                                          const int (&vend)[FQ], int j0, int s, float kscale,
-                                          QueryState *qs, uint64_t *lbase, size_t lstride,
-                                          int lane)
-{
-    uint32_t ord[FQ];
-    unsigned bal[FQ];
-    int base[FQ];
-#pragma unroll
-    for (int q = 0; q < FQ; ++q) {
-        ord[q] = ord_of_score(F[q] * kscale);
-        bal[q] = __ballot_sync(0xffffffffu, s < vend[q] && ord[q] >= bnd[q]);
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int q = 0; q < FQ; ++q)
-            base[q] = bal[q] ? atomicAdd(&qs[j0 + q].cnt, __popc(bal[q])) : 0;
-    }
-#pragma unroll
-    for (int q = 0; q < FQ; ++q) {
-        if (bal[q]) {
-            base[q] = __shfl_sync(0xffffffffu, base[q], 0);
-            if (bal[q] & (1u << lane))
-                lbase[static_cast<size_t>(j0 + q) * lstride + base[q] +
-                      __popc(bal[q] & lanemask_lt())] = make_key(ord[q], static_cast<uint32_t>(s));
-        }
-    }
-}
-
 // ------------------------------------------------------------------ generic tile math
 // One 32-column TMEM chunk: sum over the chunk's heads of w * ReLU(logit),
 // four independent accumulators.
@@ -857,6 +612,8 @@ __device__ __forceinline__ void fence_regs(uint32_t (&v)[32])
 // ------------------------------------------------------------------ epilogue
 // FC > 0: fast path for FC columns and FQ queries per warpgroup.  FC == 0:
 // generic path (kHeadsGe32 tells whether a query spans whole 32-column chunks).
+// Writes the score of every (query, key) of the item into the score buffer;
+// the selector decides what to keep.
 template <int FC, int FQ, bool kHeadsGe32>
 __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uint32_t tmem_base,
                              const WaitCtl &ctl, int wg)
@@ -866,29 +623,24 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
     const int lane = threadIdx.x & 31;
     const int bar = wg == 0 ? kBarWg0 : kBarWg1;
     const int quarter = warp & 3;             // TMEM lanes this warp may read
-    float *w_s = reinterpret_cast<float *>(smem + p.off_w);
-    QueryState *qs = reinterpret_cast<QueryState *>(smem + p.off_state);
-    WgScratch *sc = reinterpret_cast<WgScratch *>(smem + p.off_wg + wg * p.wg_bytes);
-    const uint32_t bound0 = p.mode == 1 ? 0x80000001u : 0u; // gate: score > 0
     const int j0 = wg * p.qpw;                 // first query slot this group owns
     const int col0 = j0 * p.H;                 // first TMEM column it reads
     const int ncols = p.qpw * p.H;             // TMEM columns it reads
     const int nchunk = ncols / 32;             // in 32-column chunks (generic path)
     const int cpq_shift = p.H >= 32 ? __ffs(p.H / 32) - 1 : 0;
     const int h_shift = __ffs(p.H) - 1;
-    const size_t lstride = static_cast<size_t>(p.nsplit) * p.cap;
     // the key row (of the warp's 32) whose scores this thread ends up with
     const int key_local =
         FC > 0 ? quarter * 32 + 16 * ((lane >> 1) & 1) + 8 * (lane & 1) + (lane >> 2)
                : quarter * 32 + lane;
-    int acc_use = 0;
+    int acc_use = 0, it_count = 0;
     ProfAcc pa;
     Prof pf, pt;
     const bool rec = wg == 0 && tid == 0;
     pt.start();
 
-    // Generic path: the group's weights go through shared memory, loaded into
-    // registers one item ahead.
+    // Generic path: the group's weights go through shared memory (one half
+    // per item parity), loaded into registers one item ahead.
     constexpr int kWRegs = FC > 0 ? 1 : kSlotCols / kGroupThreads;
     float wnext[kWRegs];
     if (FC == 0) {
@@ -902,27 +654,12 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
         }
     }
     float2 wr[FC > 0 ? FC / 8 : 1];
-    constexpr int CQ = FC > 0 ? FQ : 1;
-    uint32_t bnd[CQ];   // fast path: this group's admission bounds and
-    int vend[CQ];       // visibility ends, cached from qs
-
-    for (int i = tid; i < kNbCompact; i += kGroupThreads)
-        sc->hist[i] = 0;
-    named_bar_sync(bar, kGroupThreads);
 
     bool ok = true;
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
-        uint64_t *lbase = p.lists + (static_cast<size_t>(it.lrow) * p.nsplit + it.split) * p.cap;
-        for (int j = j0 + tid; j < j0 + p.qpw; j += kGroupThreads) {
-            const int i = it.q0 + j;
-            QueryState st;
-            st.cnt = 0;
-            st.bound = bound0;
-            st.vis_end = i < p.S ? visible_count(p, static_cast<long long>(i) + p.q_offset) : 0;
-            st.pad = 0;
-            qs[j] = st;
-        }
+        const int par = it_count & 1;
+        float *w_s = reinterpret_cast<float *>(smem + p.off_w) + par * p.qps * p.H;
         if constexpr (FC > 0) {
             fast_load_w<FC, FQ>(p, it, j0, lane, wr);
         } else {
@@ -941,17 +678,20 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                 }
             }
         }
-        named_bar_sync(bar, kGroupThreads);
-        if constexpr (FC > 0) {
-#pragma unroll
-            for (int q = 0; q < CQ; ++q) {
-                bnd[q] = qs[j0 + q].bound;
-                vend[q] = qs[j0 + q].vis_end;
-            }
-        }
+        // The selector must be done with this half (item it_count - 2).
+        pf.start();
+        const bool okw =
+            wait_bounded(&bars->buf_empty[par], ((it_count >> 1) & 1) ^ 1, ctl, kRoleEpilogue, id);
+        pf.add(pa, kPfEpiBufEmpty, rec);
+        ok = group_all(bar, kGroupThreads, ok && okw); // also publishes w_s
+        if (!ok)
+            break;
+        float *buf = p.scores + (static_cast<size_t>(blockIdx.x) * 2 + par) * p.qps * p.nmax +
+                     static_cast<size_t>(j0) * p.nmax;
 
-        for (int t = it.tile_begin; t < it.tile_end; ++t) {
+        for (int t = it.tile_begin; t < it.tile_end && ok; ++t) {
             const int s = t * kTileKeys + key_local;
+            const size_t off = static_cast<size_t>(t - it.tile_begin) * kTileKeys + key_local;
             float kscale = 1.0f;
             if (p.key_fp8 && s < p.T)
                 kscale = p.k_scale[static_cast<size_t>(it.b) * p.T + s];
@@ -962,99 +702,357 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
             ok = __all_sync(0xffffffffu, ok);
             pf.add(pa, kPfEpiAccFull, rec);
             pf.count(pa, kPfEpiTiles, rec);
-            if (ok) {
-                tc_fence_after();
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                       slot * kSlotCols + col0;
-                pf.start();
-                if constexpr (FC > 0) {
-                    float F[FQ];
-                    fast_tile_scores<FC, FQ>(taddr, wr, &bars->acc_empty[slot], lane, F);
-                    fast_emit<FQ>(F, bnd, vend, j0, s, kscale, qs, lbase, lstride, lane);
-                } else {
-                    // One chunk at a time, each query emitted as it completes.
-                    auto emit = [&](int jq, float score) {
-                        QueryState &st = qs[jq];
-                        const uint32_t ord = ord_of_score(score * kscale);
-                        const bool pass = s < st.vis_end && ord >= st.bound;
-                        const unsigned bal = __ballot_sync(0xffffffffu, pass);
-                        if (bal) {
-                            int base = 0;
-                            if (lane == 0)
-                                base = atomicAdd(&st.cnt, __popc(bal));
-                            base = __shfl_sync(0xffffffffu, base, 0);
-                            if (pass)
-                                lbase[static_cast<size_t>(jq) * lstride + base +
-                                      __popc(bal & lanemask_lt())] =
-                                    make_key(ord, static_cast<uint32_t>(s));
-                        }
-                    };
-                    const float *wsub = w_s + col0;
-                    float acc = 0.0f;
-                    uint32_t v[32];
-                    for (int c = 0; c < nchunk; ++c) {
-                        __syncwarp();
-                        tmem_ld_32x32b_x32(taddr + c * 32, v);
-                        tmem_ld_wait();
-                        fence_regs(v);
-                        const float *wc = wsub + c * 32;
-                        if (kHeadsGe32) {
-                            acc += chunk_dot(v, wc);
-                            if (((c + 1) & ((1 << cpq_shift) - 1)) == 0) {
-                                emit(j0 + (c >> cpq_shift), acc);
-                                acc = 0.0f;
-                            }
-                        } else {
-                            // H < 32 (a power of two): each 32-column chunk holds 32/H queries
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                acc = fmaf(fmaxf(__uint_as_float(v[i]), 0.0f), wc[i], acc);
-                                if (((i + 1) & (p.H - 1)) == 0) {
-                                    emit(j0 + ((c * 32 + i) >> h_shift), acc);
-                                    acc = 0.0f;
-                                }
-                            }
-                        }
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&bars->acc_empty[slot]);
-                }
-                pf.add(pa, kPfEpiMath, rec);
-            }
             ++acc_use;
-            pf.start();
-            ok = group_all(bar, kGroupThreads, ok);
-            pf.add(pa, kPfEpiTileBar, rec);
             if (!ok)
                 break;
-            // Cut back any list that the next tile could overflow.
-            for (int jq = j0; jq < j0 + p.qpw; ++jq) {
-                if (qs[jq].cnt > p.cap - kTileKeys) {
-                    pf.start();
-                    compact_list(p, lbase + static_cast<size_t>(jq) * lstride, qs[jq], sc, bar, tid);
-                    pf.add(pa, kPfEpiCompact, rec);
-                    pf.count(pa, kPfEpiCompactCount, rec);
-                    if constexpr (FC > 0) {
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   slot * kSlotCols + col0;
+            pf.start();
+            if constexpr (FC > 0) {
+                float F[FQ];
+                fast_tile_scores<FC, FQ>(taddr, wr, &bars->acc_empty[slot], lane, F);
 #pragma unroll
-                        for (int q = 0; q < CQ; ++q)
-                            bnd[q] = qs[j0 + q].bound;
+                for (int q = 0; q < FQ; ++q)
+                    buf[static_cast<size_t>(q) * p.nmax + off] = F[q] * kscale;
+            } else {
+                const float *wsub = w_s + col0;
+                float acc = 0.0f;
+                uint32_t v[32];
+                for (int c = 0; c < nchunk; ++c) {
+                    __syncwarp();
+                    tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    tmem_ld_wait();
+                    fence_regs(v);
+                    const float *wc = wsub + c * 32;
+                    if (kHeadsGe32) {
+                        acc += chunk_dot(v, wc);
+                        if (((c + 1) & ((1 << cpq_shift) - 1)) == 0) {
+                            buf[static_cast<size_t>(c >> cpq_shift) * p.nmax + off] = acc * kscale;
+                            acc = 0.0f;
+                        }
+                    } else {
+                        // H < 32 (a power of two): each 32-column chunk holds 32/H queries
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            acc = fmaf(fmaxf(__uint_as_float(v[i]), 0.0f), wc[i], acc);
+                            if (((i + 1) & (p.H - 1)) == 0) {
+                                buf[static_cast<size_t>((c * 32 + i) >> h_shift) * p.nmax + off] =
+                                    acc * kscale;
+                                acc = 0.0f;
+                            }
+                        }
                     }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->acc_empty[slot]);
+            }
+            pf.add(pa, kPfEpiMath, rec);
+        }
+        // Hand this half to the selector (one arrive per warp, after every
+        // lane's stores).
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&bars->buf_full[par]);
+        if (!ok)
+            *ctl.abort = 1;
+        ++it_count;
+    }
+    pt.add(pa, kPfEpiTotal, rec);
+    pa.flush(rec);
+}
+
+// ------------------------------------------------------------------ selector
+// The selector reads a query's scores in chunks of kSelChunk (16 per thread,
+// four 16-byte loads issued together), so a pass costs one memory round trip
+// per chunk.  Histogram buckets are the top 11 bits of the score's order
+// image (sign, exponent, two mantissa bits): fixed, so no range pass.
+constexpr int kSelPer = 16;
+constexpr int kSelChunk = kGroupThreads * kSelPer;   // 2048 scores
+constexpr int kSelShift = 21;                         // 2048 buckets
+
+struct SelectorScratch {
+    GroupSmall gs;
+    int out_cnt;
+    int pad[3];
+    uint32_t hist[kNbSelect];
+};
+
+// Scores base .. base+kSelChunk of sj into v (index base + 512 r + 4 tid + e
+// in v[4 r + e]); slots at or past n get the order image 0 (never kept).
+__device__ __forceinline__ void sel_load(const float *sj, int base, int n, int tid,
+                                         uint32_t (&o)[kSelPer])
+{
+    float4 x[kSelPer / 4];
+#pragma unroll
+    for (int r = 0; r < kSelPer / 4; ++r) {
+        const int i = base + r * (kGroupThreads * 4) + 4 * tid;
+        x[r] = i < n ? *reinterpret_cast<const float4 *>(sj + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < kSelPer / 4; ++r) {
+        const int i = base + r * (kGroupThreads * 4) + 4 * tid;
+        o[4 * r + 0] = i + 0 < n ? ord_of_score(x[r].x) : 0u;
+        o[4 * r + 1] = i + 1 < n ? ord_of_score(x[r].y) : 0u;
+        o[4 * r + 2] = i + 2 < n ? ord_of_score(x[r].z) : 0u;
+        o[4 * r + 3] = i + 3 < n ? ord_of_score(x[r].w) : 0u;
+    }
+}
+
+__device__ __forceinline__ int sel_index(int base, int e, int tid)
+{
+    return base + (e >> 2) * (kGroupThreads * 4) + 4 * tid + (e & 3);
+}
+
+// Appends every key of sj[0..n) (key index key0 + i) that is >= lo to `list`
+// in arbitrary order; returns how many.  One shared atomic per warp and chunk.
+__device__ int sel_emit(const float *sj, int n, int key0, uint64_t lo, uint64_t *list,
+                        SelectorScratch *sc, int tid)
+{
+    const int lane = tid & 31;
+    if (tid == 0)
+        sc->out_cnt = 0;
+    named_bar_sync(kBarSelect, kGroupThreads);
+    for (int base = 0; base < n; base += kSelChunk) {
+        uint32_t o[kSelPer];
+        sel_load(sj, base, n, tid, o);
+        uint32_t keep = 0;
+        int mine = 0;
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e) {
+            const int i = sel_index(base, e, tid);
+            const bool k = i < n && make_key(o[e], static_cast<uint32_t>(key0 + i)) >= lo;
+            keep |= k ? (1u << e) : 0u;
+            mine += k;
+        }
+        int incl = mine; // inclusive scan over the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off)
+                incl += t;
+        }
+        const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+        int wbase = 0;
+        if (lane == 0 && wtot)
+            wbase = atomicAdd(&sc->out_cnt, wtot);
+        int pos = __shfl_sync(0xffffffffu, wbase, 0) + incl - mine;
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e)
+            if (keep & (1u << e))
+                list[pos++] = make_key(o[e], static_cast<uint32_t>(key0 + sel_index(base, e, tid)));
+    }
+    named_bar_sync(kBarSelect, kGroupThreads);
+    const int c = sc->out_cnt;
+    named_bar_sync(kBarSelect, kGroupThreads); // out_cnt is reset by the next call
+    return c;
+}
+
+// Bucket of the need-th largest count in hist[0..kNbSelect) (thread tid owns
+// buckets [16 tid, 16 tid + 16)): {b*, keys above b*, keys in b*, all keys}.
+__device__ void sel_boundary(const uint32_t *hist, int need, GroupSmall *gs, int tid, int (&out)[4])
+{
+    constexpr int PER = kNbSelect / kGroupThreads;
+    const int lane = tid & 31, wid = tid >> 5;
+    uint32_t c[PER];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        c[j] = hist[tid * PER + j];
+        sum += c[j];
+    }
+    uint32_t suf = sum; // inclusive suffix sum over the warp's threads
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 32)
+            suf += t;
+    }
+    if (lane == 0)
+        gs->warp_sums[wid] = suf;
+    if (tid == 0)
+        gs->bcast[0] = -1;
+    named_bar_sync(kBarSelect, kGroupThreads);
+    uint32_t higher = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kGroupThreads / 32; ++w) {
+        higher += w > wid ? gs->warp_sums[w] : 0u;
+        total += gs->warp_sums[w];
+    }
+    const uint32_t above_thread = suf - sum + higher;
+    const uint32_t nd = static_cast<uint32_t>(need);
+    if (above_thread < nd && nd <= above_thread + sum) {
+        uint32_t above = above_thread;
+#pragma unroll
+        for (int j = PER - 1; j >= 0; --j) {
+            if (above + c[j] >= nd) {
+                gs->bcast[0] = tid * PER + j;
+                gs->bcast[1] = static_cast<int>(above);
+                gs->bcast[2] = static_cast<int>(c[j]);
+                break;
+            }
+            above += c[j];
+        }
+    }
+    named_bar_sync(kBarSelect, kGroupThreads);
+    out[0] = gs->bcast[0];
+    out[1] = gs->bcast[1];
+    out[2] = gs->bcast[2];
+    out[3] = static_cast<int>(total);
+    named_bar_sync(kBarSelect, kGroupThreads);
+}
+
+// Exact cut: the largest 64-bit key L such that exactly `need` keys with score
+// image >= lo_ord are >= L (more than `need` such keys exist; keys distinct).
+// Only for degenerate score ranges (a histogram bucket too full to keep).
+__device__ uint64_t sel_radix(const float *sj, int n, int key0, uint32_t lo_ord, int need,
+                              SelectorScratch *sc, int tid)
+{
+    const int lane = tid & 31;
+    uint64_t prefix = 0, mask = 0;
+    for (int pos = 56; pos >= 0; pos -= 8) {
+        for (int i = tid; i < 256; i += kGroupThreads)
+            sc->hist[i] = 0;
+        named_bar_sync(kBarSelect, kGroupThreads);
+        for (int base = 0; base < n; base += kSelChunk) {
+            uint32_t o[kSelPer];
+            sel_load(sj, base, n, tid, o);
+#pragma unroll
+            for (int e = 0; e < kSelPer; ++e) {
+                const int i = sel_index(base, e, tid);
+                const uint64_t key = make_key(o[e], static_cast<uint32_t>(key0 + i));
+                if (i < n && o[e] >= lo_ord && (key & mask) == prefix)
+                    atomicAdd(&sc->hist[static_cast<uint32_t>(key >> pos) & 255u], 1u);
+            }
+        }
+        named_bar_sync(kBarSelect, kGroupThreads);
+        if (tid < 32) {
+            uint32_t c[8];
+            uint32_t sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                c[j] = sc->hist[lane * 8 + j];
+                sum += c[j];
+            }
+            uint32_t suf = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
+                if (lane + off < 32)
+                    suf += t;
+            }
+            const uint32_t above_lane = suf - sum;
+            const uint32_t nd = static_cast<uint32_t>(need);
+            if (above_lane < nd && nd <= suf) {
+                uint32_t above = above_lane;
+#pragma unroll
+                for (int j = 7; j >= 0; --j) {
+                    if (above + c[j] >= nd) {
+                        sc->gs.bcast[0] = lane * 8 + j;
+                        sc->gs.bcast[1] = static_cast<int>(above);
+                        sc->gs.bcast[2] = static_cast<int>(c[j]);
+                        break;
+                    }
+                    above += c[j];
                 }
             }
         }
-        if (!ok) {
-            *ctl.abort = 1;
+        named_bar_sync(kBarSelect, kGroupThreads);
+        const int digit = sc->gs.bcast[0];
+        const int above = sc->gs.bcast[1];
+        const int inb = sc->gs.bcast[2];
+        named_bar_sync(kBarSelect, kGroupThreads);
+        need -= above;
+        prefix |= static_cast<uint64_t>(digit) << pos;
+        mask |= 0xFFull << pos;
+        if (inb == need)
             break;
-        }
-        // Publish the list lengths (rows past the end of the batch get 0).
-        for (int j = j0 + tid; j < j0 + p.qpw; j += kGroupThreads)
-            p.counts[static_cast<size_t>(it.lrow + j) * p.nsplit + it.split] =
-                j < it.nq ? qs[j].cnt : 0;
-        named_bar_sync(bar, kGroupThreads);
     }
-    pt.add(pa, kPfEpiTotal, rec);
+    return prefix;
+}
+
+// One query of a finished item: its n visible scores (keys key0..key0+n-1)
+// become a list of at most cap keys holding its top k -- all of them when
+// they fit (gated mode: all positive ones), else the keys at or above the
+// histogram bucket of the k-th largest, else exactly the top k.
+__device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint64_t *list,
+                         SelectorScratch *sc, int tid, ProfAcc &pa, bool rec)
+{
+    const uint32_t lo_ord = p.mode == 1 ? 0x80000001u : 0u; // gate: score > 0
+    const uint64_t lo_key = static_cast<uint64_t>(lo_ord) << 32;
+    if (n <= 0)
+        return 0;
+    if (n <= p.cap)
+        return sel_emit(sj, n, key0, lo_key, list, sc, tid);
+    Prof pf;
+    pf.start();
+    for (int i = tid; i < kNbSelect; i += kGroupThreads)
+        sc->hist[i] = 0;
+    named_bar_sync(kBarSelect, kGroupThreads);
+    for (int base = 0; base < n; base += kSelChunk) {
+        uint32_t o[kSelPer];
+        sel_load(sj, base, n, tid, o);
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e)
+            if (sel_index(base, e, tid) < n && o[e] >= lo_ord)
+                atomicAdd(&sc->hist[o[e] >> kSelShift], 1u);
+    }
+    named_bar_sync(kBarSelect, kGroupThreads);
+    int bd[4];
+    sel_boundary(sc->hist, p.topk, &sc->gs, tid, bd);
+    uint64_t lo;
+    if (bd[3] <= p.cap)
+        lo = lo_key;                                   // every candidate fits
+    else if (bd[1] + bd[2] <= p.cap)
+        lo = static_cast<uint64_t>(static_cast<uint32_t>(bd[0]) << kSelShift) << 32;
+    else
+        lo = sel_radix(sj, n, key0, lo_ord, p.topk, sc, tid);
+    pf.add(pa, kPfSelCut, rec);
+    return sel_emit(sj, n, key0, lo > lo_key ? lo : lo_key, list, sc, tid);
+}
+
+__device__ void run_selector(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl)
+{
+    const int tid = threadIdx.x & (kGroupThreads - 1);
+    const int lane = tid & 31;
+    SelectorScratch *sc = reinterpret_cast<SelectorScratch *>(smem + p.off_sel);
+    int it_count = 0;
+    ProfAcc pa;
+    Prof pf, pt;
+    const bool rec = tid == 0;
+    pt.start();
+    for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
+        const Item it = decode_item(p, id);
+        const int par = it_count & 1;
+        pf.start();
+        bool ok = wait_bounded(&bars->buf_full[par], (it_count >> 1) & 1, ctl, kRoleSelect, id);
+        ok = group_all(kBarSelect, kGroupThreads, ok);
+        pf.add(pa, kPfSelBufFull, rec);
+        if (!ok)
+            break;
+        pf.start();
+        const float *buf = p.scores + (static_cast<size_t>(blockIdx.x) * 2 + par) * p.qps * p.nmax;
+        const int key0 = it.tile_begin * kTileKeys;
+        const int key_end = it.tile_end * kTileKeys;
+        for (int j = 0; j < it.nq; ++j) {
+            const int vis = visible_count(p, static_cast<long long>(it.q0 + j) + p.q_offset);
+            const int n = max(0, min(vis, key_end) - key0);
+            uint64_t *list = p.lists + (static_cast<size_t>(it.lrow + j) * p.nsplit + it.split) * p.cap;
+            const int c = sel_query(p, buf + static_cast<size_t>(j) * p.nmax, n, key0, list, sc, tid,
+                                    pa, rec);
+            if (tid == 0)
+                p.counts[static_cast<size_t>(it.lrow + j) * p.nsplit + it.split] = c;
+        }
+        // every read of this half is done
+        named_bar_sync(kBarSelect, kGroupThreads);
+        pf.add(pa, kPfSelBusy, rec);
+        if (lane == 0)
+            mbar_arrive(&bars->buf_empty[par]);
+        ++it_count;
+    }
+    pt.add(pa, kPfSelTotal, rec);
     pa.flush(rec);
 }
 
@@ -1086,6 +1084,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->acc_full[s], 1);
             mbar_init(&bars->acc_empty[s], epi_warps);
+            mbar_init(&bars->buf_full[s], epi_warps);
+            mbar_init(&bars->buf_empty[s], kGroupThreads / 32);
         }
         bars->abort = 0;
         fence_mbar_init();
@@ -1107,7 +1107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wg = warp >> 2;
         if (wg < p.n_wg)
             run_epilogue<FC, FQ, kHeadsGe32>(p, smem, bars, tmem_base, ctl, wg);
-    } else {
+    } else if (warp < 12) {
         regs_dec<kCtlRegs>();
         if (warp == 8 && lane == 0)
             run_producer(p, &tmQ, &tmK, smem, bars, ctl);
@@ -1115,6 +1115,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             run_mma(p, smem, bars, tmem_base, ctl);
         else if (warp >= 10 && p.key_fp8)
             run_converter(p, smem, bars, ctl, threadIdx.x - 320);
+    } else {
+        regs_dec<kCtlRegs>();
+        run_selector(p, smem, bars, ctl);
     }
 
     tc_fence_before();
