@@ -14,15 +14,15 @@
 //      that in total first go through a radix select over the 64-bit keys,
 //      read from global memory one byte per pass, which finds the k-th largest
 //      key L; the k keys >= L are gathered.
-//   2. A histogram over NB buckets linear in the score, spanning the keys' own
-//      [min, max], finds the bucket holding the k-th largest key; the keys of
+//   2. A histogram over NB buckets spanning the keys' own [min, max] (integer
+//      ranges of the score image when all scores share a sign, else linear in
+//      the score) finds the bucket holding the k-th largest key; the keys of
 //      that bucket and above are scattered into bucket order (a counting
 //      sort); each key is then ranked among the keys of its own bucket and
-//      moved to its final slot (the buckets average a few keys).  A bucket too
-//      full for that -- many equal or near-equal scores -- sends the row to a
-//      bitonic sort instead.
-//   3. The first min(k, n) keys become (index, score) pairs; the rest of the
-//      row is padded with (-1, -inf).
+//      written straight to its output slot (the buckets average a few keys).
+//      A bucket too full for that -- many equal or near-equal scores -- sends
+//      the row to a bitonic sort instead.
+//   3. The slots past min(k, n) are padded with (-1, -inf).
 // While a row is processed, the next row's list is prefetched into L2.
 #pragma once
 #include <cstdint>
@@ -56,7 +56,7 @@ struct SelSmem {
     int misc[4];
     uint32_t hist[kSelNb];
     uint64_t out[kSelKeys];
-    uint64_t top[kMaxTopk];   // the sorted top k (fast path)
+    uint16_t out_b[kSelKeys]; // bucket of out[i] (fast path)
 };
 
 __device__ __forceinline__ void sel_prefetch_l2(const void *src, uint32_t bytes)
@@ -132,11 +132,33 @@ __device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_li
     return prefix;
 }
 
-// Sorts the n keys of e[] (0 = empty slot, n <= kSelKeys): returns a shared
-// buffer holding the top `kept` of them (kept <= n) in descending order at
-// [0, kept).
-__device__ const uint64_t *sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEpt], int n,
-                                         int kept, int tid)
+// Bucket of a score image: integer ranges of the image when every key has the
+// same sign (the image is then roughly logarithmic in the score, which spreads
+// the dense scores just above a cut), linear in the score otherwise.
+struct SelMap {
+    uint32_t mn;
+    int shift;
+    bool by_ord;
+    BucketMap bm;
+};
+
+__device__ __forceinline__ int sel_bucket(uint32_t o, const SelMap &m)
+{
+    if (m.by_ord)
+        return kSelNb - 1 - static_cast<int>((o - m.mn) >> m.shift);
+    return kSelNb - 1 - bucket_of(score_of_ord(o), m.bm, kSelNb);
+}
+
+__device__ __forceinline__ void sel_store(int32_t *oi, float *os, int slot, uint64_t key)
+{
+    oi[slot] = key_index(key);
+    os[slot] = key_score(key);
+}
+
+// Writes the top `kept` (kept <= n) of the n keys of e[] (0 = empty slot,
+// n <= kSelKeys) in descending order to oi/os[0..kept).
+__device__ void sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEpt], int n, int kept, int tid,
+                              int32_t *oi, float *os)
 {
     const int lane = tid & 31, wid = tid >> 5;
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
@@ -162,15 +184,20 @@ __device__ const uint64_t *sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEp
         mn = min(mn, sm->gs.warp_sums[w]);
         mx = max(mx, sm->gs.warp_sums[16 + w]);
     }
-    const BucketMap bm = bucket_map(mn, mx, kSelNb);
+    SelMap map;
+    map.mn = mn;
+    map.by_ord = (mn >> 31) == (mx >> 31);
+    const uint32_t span = mx - mn;
+    map.shift = span < static_cast<uint32_t>(kSelNb) ? 0 : 32 - __clz(span) - 11;
+    map.bm = bucket_map(mn, mx, kSelNb);
     int total = n;
-    bool fallback = !bm.ok;
+    bool fallback = mx == mn || (!map.by_ord && !map.bm.ok);
     if (!fallback) {
         // histogram, buckets numbered from the top score down
         int db[kSelEpt];
 #pragma unroll
         for (int i = 0; i < kSelEpt; ++i) {
-            db[i] = e[i] != 0 ? kSelNb - 1 - bucket_of(key_score(e[i]), bm, kSelNb) : kSelNb;
+            db[i] = e[i] != 0 ? sel_bucket(key_ord(e[i]), map) : kSelNb;
             if (db[i] < kSelNb)
                 atomicAdd(&sm->hist[db[i]], 1u);
         }
@@ -225,9 +252,13 @@ __device__ const uint64_t *sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEp
             big = max(big, static_cast<int>(sm->gs.warp_sums[w]));
         // scatter the keys of buckets <= db* into bucket order
 #pragma unroll
-        for (int i = 0; i < kSelEpt; ++i)
-            if (db[i] <= dstar)
-                sm->out[atomicAdd(&sm->hist[db[i]], 1u)] = e[i];
+        for (int i = 0; i < kSelEpt; ++i) {
+            if (db[i] <= dstar) {
+                const uint32_t slot = atomicAdd(&sm->hist[db[i]], 1u);
+                sm->out[slot] = e[i];
+                sm->out_b[slot] = static_cast<uint16_t>(db[i]);
+            }
+        }
         __syncthreads();
         if (big <= kSelSmallBucket) {
             // Rank each placed key inside its bucket (keys are distinct) and
@@ -236,17 +267,16 @@ __device__ const uint64_t *sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEp
             // a warp see buckets of similar size.
             for (int a = tid; a < total; a += kSelThreads) {
                 const uint64_t x = sm->out[a];
-                const int b = kSelNb - 1 - bucket_of(key_score(x), bm, kSelNb);
+                const int b = sm->out_b[a];
                 const int lo_s = b == 0 ? 0 : static_cast<int>(sm->hist[b - 1]);
                 const int hi_s = static_cast<int>(sm->hist[b]);
                 int to = lo_s;
                 for (int j = lo_s; j < hi_s; ++j)
                     to += sm->out[j] > x ? 1 : 0;
                 if (to < kept)
-                    sm->top[to] = x;
+                    sel_store(oi, os, to, x);
             }
-            __syncthreads();
-            return sm->top;
+            return;
         }
     } else {
         // degenerate range (one score for every key): all keys to out[]
@@ -268,7 +298,8 @@ __device__ const uint64_t *sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEp
         sm->out[i] = 0ull;
     __syncthreads();
     bitonic_sort_desc<kSelThreads>(sm->out, P, 0, tid);
-    return sm->out;
+    for (int i = tid; i < kept; i += kSelThreads)
+        sel_store(oi, os, i, sm->out[i]);
 }
 
 constexpr int kSelCtasPerSm = 3;
@@ -371,18 +402,13 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
             __syncthreads(); // out[] is rewritten below
         }
         const int kept = min(n, sp.topk);
-        const uint64_t *res = kept > 0 ? sel_sort_regs(sm, e, n, kept, tid) : sm->out;
         int32_t *oi = sp.out_idx + orow * sp.topk;
         float *os = sp.out_score + orow * sp.topk;
-        for (int i = tid; i < sp.topk; i += kSelThreads) {
-            if (i < kept) {
-                const uint64_t key = res[i];
-                oi[i] = key_index(key);
-                os[i] = key_score(key);
-            } else {
-                oi[i] = -1;
-                os[i] = -__int_as_float(0x7f800000);
-            }
+        if (kept > 0)
+            sel_sort_regs(sm, e, n, kept, tid, oi, os);
+        for (int i = kept + tid; i < sp.topk; i += kSelThreads) {
+            oi[i] = -1;
+            os[i] = -__int_as_float(0x7f800000);
         }
         __syncthreads();
     }
