@@ -77,6 +77,19 @@ def measured_traffic(config: str, sha: str):
     return None
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest of every rank's value (the job is as slow as its slowest
+    rank); the value itself on a single process."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -327,11 +340,7 @@ def main():
                 for row in marks]
     select_ms = [sum(row[2 * c + 1].elapsed_time(row[2 * c + 2])
                      for c in range(plan.launches // 2)) for row in marks]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     queries = wl.B * wl.S
     value = queries * world / (ms_per_step / 1000.0)
@@ -374,11 +383,7 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
         e2e = {"value": queries * world / (e_ms / 1000.0), "unit": "queries/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms}
