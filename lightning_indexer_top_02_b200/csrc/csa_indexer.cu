@@ -179,6 +179,11 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     // whole 32-column TMEM loads.
     p.n_wg = (qps >= 2 && p.N >= 64) ? 2 : 1;
     p.qpw = qps / p.n_wg;
+    // One query per item: both warpgroups read every column and take
+    // alternate key tiles instead of splitting the queries.
+    p.tile_split = qps == 1 ? 1 : 0;
+    if (p.tile_split)
+        p.n_wg = 2;
 
     // Candidate list per (query, split): the top k plus room for the
     // selector's histogram bucket around the k-th score.
@@ -187,30 +192,48 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
         extra = 256;
     p.cap = (p.topk + extra + 127) / 128 * 128;
 
-    // per pipeline stage: the MMA's 16-bit key tile, plus (E4M3 keys) the raw
-    // staged tile it is converted from
-    const int k_stage = csa::kTileKeys * p.d * 2 + (p.key_fp8 ? csa::kTileKeys * p.d : 0);
+    // Key tiles: the MMA's ring of 16-bit tiles, plus (E4M3 keys) a staging
+    // ring of raw tiles that the TMA fills.  E4M3 staging gets what is left
+    // after four (small query blocks, where short MMAs make every hand-off
+    // count) or three 16-bit stages.
+    const int k16 = csa::kTileKeys * p.d * 2;
+    const int k8 = csa::kTileKeys * p.d;
     int off = 0;
     p.off_q = off;
     off += p.N * p.d * 2;
     p.off_k = off;
     int tail = 0;
-    tail += 2 * p.qps * p.H * 4;                               // w, one half per item parity
+    tail += 4 * p.qps * p.H * 4;                               // w: per item parity (and group)
     tail = (tail + 15) / 16 * 16;
     tail += (static_cast<int>(sizeof(csa::SelectorScratch)) + 15) / 16 * 16;
     tail += static_cast<int>(sizeof(csa::Barriers)) + 16;
-    int stages = (kSmemLimit - 1024 - off - tail) / k_stage;
-    if (stages > csa::kMaxStages)
-        stages = csa::kMaxStages;
-    if (stages < 2)
-        return CSA_ERR_UNSUPPORTED;
+    const int room = kSmemLimit - 1024 - off - tail;
+    int stages, stages8 = 0;
+    if (p.key_fp8) {
+        stages = p.N <= 64 ? 4 : 3;
+        stages8 = (room - stages * k16) / k8;
+        if (stages8 > csa::kMaxStages)
+            stages8 = csa::kMaxStages;
+        if (stages8 < 2) {
+            stages = 2;
+            stages8 = (room - stages * k16) / k8;
+        }
+        if (stages8 < 2)
+            return CSA_ERR_UNSUPPORTED;
+    } else {
+        stages = room / k16;
+        if (stages > csa::kMaxStages)
+            stages = csa::kMaxStages;
+        if (stages < 2)
+            return CSA_ERR_UNSUPPORTED;
+    }
     p.stages = stages;
-    off += stages * csa::kTileKeys * p.d * 2;
+    p.stages8 = stages8;
+    off += stages * k16;
     p.off_k8 = off;
-    if (p.key_fp8)
-        off += stages * csa::kTileKeys * p.d;
+    off += stages8 * k8;
     p.off_w = off;
-    off += 2 * p.qps * p.H * 4;
+    off += 4 * p.qps * p.H * 4;
     off = (off + 15) / 16 * 16;
     p.off_sel = off;
     off += (static_cast<int>(sizeof(csa::SelectorScratch)) + 15) / 16 * 16;

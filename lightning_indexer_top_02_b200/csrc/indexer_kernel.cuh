@@ -133,12 +133,14 @@ struct Params {
     int qps;      // queries per item
     int N;        // MMA N = qps * H (<= 256)
     int n_wg;     // epilogue warpgroups in use (1 or 2)
-    int qpw;      // queries per epilogue warpgroup = qps / n_wg
+    int qpw;      // queries per epilogue warpgroup = qps / n_wg (or qps when tile_split)
+    int tile_split; // one query per item: both warpgroups take every column, alternate tiles
     int qb_lo;    // first query block (per batch) of this launch
     int nqb;      // query blocks per batch in this launch
     int nsplit;   // key-range splits per query block
     int n_items;
-    int stages;
+    int stages;   // 16-bit key tiles in the MMA's ring
+    int stages8;  // E4M3 keys: raw tiles in the staging ring
     int cap;      // candidate list capacity per query and split
     int nmax;     // score-buffer keys per query (the longest item's key range)
     int row_bytes;   // bytes of one swizzled operand row: min(128, 2*d)
@@ -262,12 +264,12 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
             }
         }
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
-            const int stage = kload % p.stages;
             const int row = it.b * p.T + t * kTileKeys;
             pf.start();
             if (p.key_fp8) {
                 // raw E4M3 tile (128 rows x d bytes) into the staging ring
-                if (!wait_bounded(&bars->k8_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
+                const int stage = kload % p.stages8;
+                if (!wait_bounded(&bars->k8_empty[stage], ((kload / p.stages8) & 1) ^ 1, ctl,
                                   kRoleProducer, id))
                     goto unwind;
                 pf.add(pa, kPfProdKEmpty, true);
@@ -275,6 +277,7 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
                 tma_load_2d(smem + p.off_k8 + stage * kTileKeys * p.d, tmK, &bars->k8_full[stage],
                             0, row);
             } else {
+                const int stage = kload % p.stages;
                 if (!wait_bounded(&bars->k_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
                                   kRoleProducer, id))
                     goto unwind;
@@ -290,9 +293,10 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
     }
 unwind:
     // Let every copy already issued land before the CTA can exit.
-    for (int s = 0; s < p.stages; ++s) {
+    const int ring = p.key_fp8 ? p.stages8 : p.stages;
+    for (int s = 0; s < ring; ++s) {
         if (kload > s) {
-            const int fills = (kload - s + p.stages - 1) / p.stages;
+            const int fills = (kload - s + ring - 1) / ring;
             wait_drain(p.key_fp8 ? &bars->k8_full[s] : &bars->k_full[s], (fills - 1) & 1);
         }
     }
@@ -453,15 +457,16 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
             mbar_arrive(&bars->q_ready);
         ++quse;
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
-            const int stage = kuse % p.stages;
-            const uint32_t par = (kuse / p.stages) & 1;
-            ok = wait_bounded(&bars->k8_full[stage], par, ctl, kRoleConvert, id);
-            ok = ok && wait_bounded(&bars->k_empty[stage], par ^ 1, ctl, kRoleConvert, id);
+            const int stage = kuse % p.stages;      // slot in the f16 ring
+            const int stage8 = kuse % p.stages8;    // slot in the staging ring
+            ok = wait_bounded(&bars->k8_full[stage8], (kuse / p.stages8) & 1, ctl, kRoleConvert, id);
+            ok = ok && wait_bounded(&bars->k_empty[stage], ((kuse / p.stages) & 1) ^ 1, ctl,
+                                    kRoleConvert, id);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 return;
             const uint4 *src =
-                reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage * kTileKeys * p.d);
+                reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage8 * kTileKeys * p.d);
             uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
 #pragma unroll
             for (int i = 0; i < kConvUnits; ++i) {
@@ -479,7 +484,7 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bars->k_full[stage]);
-                mbar_arrive(&bars->k8_empty[stage]);
+                mbar_arrive(&bars->k8_empty[stage8]);
             }
             ++kuse;
         }
@@ -623,7 +628,7 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
     const int lane = threadIdx.x & 31;
     const int bar = wg == 0 ? kBarWg0 : kBarWg1;
     const int quarter = warp & 3;             // TMEM lanes this warp may read
-    const int j0 = wg * p.qpw;                 // first query slot this group owns
+    const int j0 = p.tile_split ? 0 : wg * p.qpw; // first query slot this group owns
     const int col0 = j0 * p.H;                 // first TMEM column it reads
     const int ncols = p.qpw * p.H;             // TMEM columns it reads
     const int nchunk = ncols / 32;             // in 32-column chunks (generic path)
@@ -634,13 +639,15 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
         FC > 0 ? quarter * 32 + 16 * ((lane >> 1) & 1) + 8 * (lane & 1) + (lane >> 2)
                : quarter * 32 + lane;
     int acc_use = 0, it_count = 0;
+    int gtile = 0; // tiles of this CTA so far (tile_split: even ones are group 0's)
     ProfAcc pa;
     Prof pf, pt;
     const bool rec = wg == 0 && tid == 0;
     pt.start();
 
     // Generic path: the group's weights go through shared memory (one half
-    // per item parity), loaded into registers one item ahead.
+    // per item parity; per group when tile_split), loaded into registers one
+    // item ahead.
     constexpr int kWRegs = FC > 0 ? 1 : kSlotCols / kGroupThreads;
     float wnext[kWRegs];
     if (FC == 0) {
@@ -659,7 +666,10 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         const int par = it_count & 1;
-        float *w_s = reinterpret_cast<float *>(smem + p.off_w) + par * p.qps * p.H;
+        // tile_split: both groups use every column, so each has its own halves
+        // (a group can run up to two items ahead of the other)
+        float *w_s = reinterpret_cast<float *>(smem + p.off_w) +
+                     ((p.tile_split ? wg : 0) * 2 + par) * p.qps * p.H;
         if constexpr (FC > 0) {
             fast_load_w<FC, FQ>(p, it, j0, lane, wr);
         } else {
@@ -690,14 +700,18 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                      static_cast<size_t>(j0) * p.nmax;
 
         for (int t = it.tile_begin; t < it.tile_end && ok; ++t) {
+            if (p.tile_split && (gtile++ & 1) != wg)
+                continue;                            // the other group's tile
             const int s = t * kTileKeys + key_local;
             const size_t off = static_cast<size_t>(t - it.tile_begin) * kTileKeys + key_local;
             float kscale = 1.0f;
             if (p.key_fp8 && s < p.T)
                 kscale = p.k_scale[static_cast<size_t>(it.b) * p.T + s];
-            const int slot = acc_use & 1;
+            // tile_split: group w always drains slot w, every use flips its phase
+            const int slot = p.tile_split ? wg : acc_use & 1;
+            const uint32_t par = p.tile_split ? (acc_use & 1) : ((acc_use >> 1) & 1);
             pf.start();
-            ok = wait_bounded(&bars->acc_full[slot], (acc_use >> 1) & 1, ctl, kRoleEpilogue, id);
+            ok = wait_bounded(&bars->acc_full[slot], par, ctl, kRoleEpilogue, id);
             // the TMEM loads below are warp-collective: agree on the outcome first
             ok = __all_sync(0xffffffffu, ok);
             pf.add(pa, kPfEpiAccFull, rec);
@@ -1078,12 +1092,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&bars->k_full[s], p.key_fp8 ? 2 : 1); // converters, or the TMA's tx
             mbar_init(&bars->k_empty[s], 1);
+        }
+        for (int s = 0; s < p.stages8; ++s) {
             mbar_init(&bars->k8_full[s], 1);
             mbar_init(&bars->k8_empty[s], 2);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->acc_full[s], 1);
-            mbar_init(&bars->acc_empty[s], epi_warps);
+            mbar_init(&bars->acc_empty[s], p.tile_split ? 4 : epi_warps);
             mbar_init(&bars->buf_full[s], epi_warps);
             mbar_init(&bars->buf_empty[s], kGroupThreads / 32);
         }

@@ -11,9 +11,11 @@
 //
 // One CTA of 256 threads per query row at a time, several CTAs per SM:
 //   1. The row's keys go to registers (16 per thread).  Lists longer than
-//      that in total first go through a radix select over the 64-bit keys,
-//      read from global memory one byte per pass, which finds the k-th largest
-//      key L; the k keys >= L are gathered.
+//      that in total (key-range splits) first go through one histogram pass
+//      over the lists in global memory, and the keys at or above the bucket of
+//      the k-th largest are gathered; if that bucket is too full, a radix
+//      select over the 64-bit keys (one byte per pass) finds the k-th largest
+//      key L exactly and the k keys >= L are gathered.
 //   2. A histogram over NB buckets spanning the keys' own [min, max] (integer
 //      ranges of the score image when all scores share a sign, else linear in
 //      the score) finds the bucket holding the k-th largest key; the keys of
@@ -64,6 +66,68 @@ __device__ __forceinline__ void sel_prefetch_l2(const void *src, uint32_t bytes)
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
                  "r"(bytes)
                  : "memory");
+}
+
+// For rows whose lists hold more keys than fit in registers: one histogram
+// pass over the lists in global memory (buckets = top 11 bits of the score
+// image) finds the bucket of the k-th largest key; returns the key L such that
+// every key >= L is at or above that bucket, with *count keys >= L.
+__device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *row_lists,
+                                         SelSmem *sm, int tid, int *count)
+{
+    const int lane = tid & 31, wid = tid >> 5;
+    for (int i = tid; i < kSelNb; i += kSelThreads)
+        sm->hist[i] = 0;
+    __syncthreads();
+    for (int s = 0; s < sp.nsplit; ++s) {
+        const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
+        const int n = sm->split_off[s + 1] - sm->split_off[s];
+        for (int j = tid; j < n; j += kSelThreads)
+            atomicAdd(&sm->hist[key_ord(src[j]) >> 21], 1u);
+    }
+    __syncthreads();
+    // bucket of the k-th largest, top bucket first
+    constexpr int PER = kSelNb / kSelThreads;
+    uint32_t c[PER];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        c[j] = sm->hist[tid * PER + j];
+        sum += c[j];
+    }
+    uint32_t suf = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 32)
+            suf += t;
+    }
+    if (lane == 0)
+        sm->gs.warp_sums[wid] = suf;
+    __syncthreads();
+    uint32_t higher = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w)
+        higher += w > wid ? sm->gs.warp_sums[w] : 0u;
+    const uint32_t above_thread = suf - sum + higher;
+    const uint32_t nd = static_cast<uint32_t>(sp.topk);
+    if (above_thread < nd && nd <= above_thread + sum) {
+        uint32_t above = above_thread;
+#pragma unroll
+        for (int j = PER - 1; j >= 0; --j) {
+            if (above + c[j] >= nd) {
+                sm->misc[0] = tid * PER + j;
+                sm->misc[1] = static_cast<int>(above + c[j]);
+                break;
+            }
+            above += c[j];
+        }
+    }
+    __syncthreads();
+    *count = sm->misc[1];
+    const uint64_t L = static_cast<uint64_t>(static_cast<uint32_t>(sm->misc[0]) << 21) << 32;
+    __syncthreads();
+    return L;
 }
 
 // Radix select over the row's lists in global memory: the largest L such that
@@ -358,7 +422,14 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
         int n = n_all;
         uint64_t e[kSelEpt];
         if (n_all > kSelKeys) {
-            const uint64_t L = sel_radix_global(sp, row_lists, sm, sp.topk, tid);
+            // keys at or above the histogram bucket of the k-th largest; an
+            // exact radix cut when that bucket is too full
+            int kept_pre;
+            uint64_t L = sel_prefilter_global(sp, row_lists, sm, tid, &kept_pre);
+            if (kept_pre > kSelKeys)
+                L = sel_radix_global(sp, row_lists, sm, sp.topk, tid);
+            else
+                n = kept_pre;
             if (tid == 0)
                 sm->misc[2] = 0;
             __syncthreads();
@@ -372,7 +443,8 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
                 }
             }
             __syncthreads();
-            n = sp.topk;
+            if (n == n_all)
+                n = sp.topk; // the radix cut keeps exactly k
 #pragma unroll
             for (int i = 0; i < kSelEpt; ++i) {
                 const int j = i * kSelThreads + tid;
