@@ -238,8 +238,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=512,
                     help="query rows of the CPU-baseline sample (rank 0)")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
-                    help="override a workload field (B, S, T, H, d, m, topk, seed, key_fp8, "
-                         "gated), e.g. for a reduced profiling shape; the workload name records it")
+                    help="override a workload field (B, S, T, H, d, m, topk, seed, causal, "
+                         "key_fp8, gated), e.g. for a reduced profiling shape; the workload name records it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -249,9 +249,11 @@ def main():
         kw = {}
         for item in args.set:
             field, _, value = item.partition("=")
-            if field not in ("B", "S", "T", "H", "d", "m", "topk", "seed", "key_fp8", "gated"):
+            if field not in ("B", "S", "T", "H", "d", "m", "topk", "seed", "causal", "key_fp8",
+                             "gated"):
                 raise SystemExit(f"--set: unknown field {field!r}")
-            kw[field] = (value.lower() in ("1", "true")) if field in ("key_fp8", "gated") else int(value)
+            flag = field in ("causal", "key_fp8", "gated")
+            kw[field] = (value.lower() in ("1", "true")) if flag else int(value)
         wl = wl.replace(name=wl.name + "[" + ",".join(args.set) + "]", **kw)
 
     if args.impl == "reference":

@@ -77,7 +77,8 @@ enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelec
 enum ProfSlot : int {
     kPfProdQEmpty, kPfProdKEmpty, kPfMmaQFull, kPfMmaKFull, kPfMmaAccEmpty, kPfMmaTotal,
     kPfEpiAccFull, kPfEpiBufEmpty, kPfEpiTotal, kPfEpiTiles, kPfEpiMath, kPfSelBufFull,
-    kPfSelBusy, kPfSelTotal, kPfSelCut, kPfSlots
+    kPfSelBusy, kPfSelTotal, kPfSelCut, kPfCvtK8Full, kPfCvtKEmpty, kPfCvtWork, kPfCvtTotal,
+    kPfSlots
 };
 #ifdef CSA_PROFILE
 constexpr int kProfCtas = 160;
@@ -434,6 +435,10 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
         }
     }
     const uint32_t dst_step = static_cast<uint32_t>(kConvThreads / units_per_row * p.row_bytes);
+    ProfAcc pa;
+    Prof pf, pt;
+    const bool rec = ct == 0;
+    pt.start();
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         bool ok = wait_bounded(&bars->q_full, quse & 1, ctl, kRoleConvert, id);
@@ -459,12 +464,17 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
             const int stage = kuse % p.stages;      // slot in the f16 ring
             const int stage8 = kuse % p.stages8;    // slot in the staging ring
+            pf.start();
             ok = wait_bounded(&bars->k8_full[stage8], (kuse / p.stages8) & 1, ctl, kRoleConvert, id);
+            pf.add(pa, kPfCvtK8Full, rec);
+            pf.start();
             ok = ok && wait_bounded(&bars->k_empty[stage], ((kuse / p.stages) & 1) ^ 1, ctl,
                                     kRoleConvert, id);
+            pf.add(pa, kPfCvtKEmpty, rec);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 return;
+            pf.start();
             const uint4 *src =
                 reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage8 * kTileKeys * p.d);
             uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
@@ -486,9 +496,12 @@ __device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, co
                 mbar_arrive(&bars->k_full[stage]);
                 mbar_arrive(&bars->k8_empty[stage8]);
             }
+            pf.add(pa, kPfCvtWork, rec);
             ++kuse;
         }
     }
+    pt.add(pa, kPfCvtTotal, rec);
+    pa.flush(rec);
 }
 
 // ------------------------------------------------------------------ fast tile math
