@@ -192,48 +192,36 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
         extra = 256;
     p.cap = (p.topk + extra + 127) / 128 * 128;
 
-    // Key tiles: the MMA's ring of 16-bit tiles, plus (E4M3 keys) a staging
-    // ring of raw tiles that the TMA fills.  E4M3 staging gets what is left
-    // after four (small query blocks, where short MMAs make every hand-off
-    // count) or three 16-bit stages.
-    const int k16 = csa::kTileKeys * p.d * 2;
-    const int k8 = csa::kTileKeys * p.d;
+    // Shared memory: the bf16 query block (where the TMA lands it), with E4M3
+    // keys its two E4M3 pieces (hi8 and lo8 blocks of N rows x d bytes), the
+    // ring of key tiles (bf16, or E4M3 as stored) with every stage that fits,
+    // then weights, query scales, selector scratch and barriers.
+    const int ktile = csa::kTileKeys * p.d * (p.key_fp8 ? 1 : 2);
     int off = 0;
     p.off_q = off;
     off += p.N * p.d * 2;
+    if (p.key_fp8) {
+        p.off_e = off;
+        off += 2 * p.N * p.d;
+    }
     p.off_k = off;
-    int tail = 0;
-    tail += 4 * p.qps * p.H * 4;                               // w: per item parity (and group)
-    tail = (tail + 15) / 16 * 16;
+    const int w_bytes = 4 * p.qps * p.H * 4;           // w: per item parity (and group)
+    const int sig_bytes = p.key_fp8 ? 2 * p.N * 4 : 0;  // query scales: per item parity
+    int tail = (w_bytes + sig_bytes + 15) / 16 * 16;
     tail += (static_cast<int>(sizeof(csa::SelectorScratch)) + 15) / 16 * 16;
     tail += static_cast<int>(sizeof(csa::Barriers)) + 16;
     const int room = kSmemLimit - 1024 - off - tail;
-    int stages, stages8 = 0;
-    if (p.key_fp8) {
-        stages = p.N <= 64 ? 4 : 3;
-        stages8 = (room - stages * k16) / k8;
-        if (stages8 > csa::kMaxStages)
-            stages8 = csa::kMaxStages;
-        if (stages8 < 2) {
-            stages = 2;
-            stages8 = (room - stages * k16) / k8;
-        }
-        if (stages8 < 2)
-            return CSA_ERR_UNSUPPORTED;
-    } else {
-        stages = room / k16;
-        if (stages > csa::kMaxStages)
-            stages = csa::kMaxStages;
-        if (stages < 2)
-            return CSA_ERR_UNSUPPORTED;
-    }
+    int stages = room / ktile;
+    if (stages > csa::kMaxStages)
+        stages = csa::kMaxStages;
+    if (stages < 2)
+        return CSA_ERR_UNSUPPORTED;
     p.stages = stages;
-    p.stages8 = stages8;
-    off += stages * k16;
-    p.off_k8 = off;
-    off += stages8 * k8;
+    off += stages * ktile;
     p.off_w = off;
-    off += 4 * p.qps * p.H * 4;
+    off += w_bytes;
+    p.off_sig = off;
+    off += sig_bytes;
     off = (off + 15) / 16 * 16;
     p.off_sel = off;
     off += (static_cast<int>(sizeof(csa::SelectorScratch)) + 15) / 16 * 16;
@@ -390,9 +378,12 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
                    p.N, swz))
         return CSA_ERR_CUDA;
     if (p.key_fp8) {
-        // raw E4M3 rows, unswizzled: the converters rewrite them swizzled
+        // E4M3 rows of d bytes, swizzled at that width: the MMA's A operand as is
+        const CUtensorMapSwizzle swz8 = p.d == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                        : p.d == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_32B;
         if (!make_tmap(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->k, static_cast<long long>(p.B) * p.T,
-                       p.d, p.d, csa::kTileKeys, CU_TENSOR_MAP_SWIZZLE_NONE, 1))
+                       p.d, p.d, csa::kTileKeys, swz8, 1))
             return CSA_ERR_CUDA;
     } else if (!make_tmap(&tmK, qdt, a->k, static_cast<long long>(p.B) * p.T, p.d,
                           p.row_bytes / 2, csa::kTileKeys, swz)) {

@@ -23,15 +23,14 @@
 //   warp 8       TMA producer: the query block once per item (with an L2
 //                prefetch of the next item's), key tiles into a ring
 //   warp 9       TMEM owner and MMA issuer (one thread): per key tile, d/16
-//                tcgen05.mma (M = 128 keys, N = qps*H_I) into one of two
-//                256-column TMEM accumulators
-//   warps 10,11  E4M3 keys only: converters.  The producer lands each FP8 key
-//                tile in a staging ring; the converters rewrite it as f16
-//                into the MMA's swizzled key ring (exact: every E4M3 value is
-//                an f16 normal) and convert the item's query block from bf16
-//                to f16 in place (exact for |q| < 65504), so the MMA runs
-//                kind::f16 with both operands f16.  The key's fp32 scale
-//                multiplies its score after the head reduction (scale > 0).
+//                tcgen05.mma kind::f16 (M = 128 keys, N = qps*H_I) into one
+//                of two 256-column TMEM accumulators; with E4M3 keys, 2*d/32
+//                kind::f8f6f4 MMAs (the key tile as stored, times the two
+//                E4M3 pieces of the query block, summed in one accumulator)
+//   warps 10,11  E4M3 keys only: query splitter.  Each item's bf16 query rows
+//                become sigma * (hi8 + lo8) (run_qsplit); sigma folds into the
+//                head weights and the key's fp32 scale multiplies its score
+//                after the head reduction (both scales > 0).
 //   warps 12..15 selector
 // The block launches with 128 registers per thread; the two control
 // warpgroups give most of their share to the epilogue warpgroups
@@ -60,25 +59,25 @@ constexpr int kSlotCols = 256;   // TMEM columns per accumulator slot
 constexpr int kThreads = 512;
 constexpr int kLaunchRegs = 128;  // registers per thread the kernel must be built with
 constexpr int kEpiRegs = 160;     // after the split: epilogue warpgroups
-constexpr int kCtlRegs = 96;      //                  producer / MMA / converters, selector
+constexpr int kCtlRegs = 96;      //                  producer / MMA / splitter, selector
 static_assert(2 * 128 * kEpiRegs + 2 * 128 * kCtlRegs == kThreads * kLaunchRegs,
               "register split must match the launch budget");
 constexpr int kGroupThreads = 128;
 constexpr int kBarWg0 = 1, kBarWg1 = 2, kBarSelect = 3;  // named barriers
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kMaxTopk = 2048;
 constexpr int kNbSelect = 2048;  // buckets of the selector's histogram
 constexpr int kMaxItemKeys = 65536; // keys of one work item (longer ranges are split)
 
-enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelect = 4, kRoleConvert = 5 };
+enum Role : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleSelect = 4, kRoleSplit = 5 };
 
 // Optional per-role cycle counters (built only with -DCSA_PROFILE): where each
 // role spends its time, recorded by one thread per role and CTA.
 enum ProfSlot : int {
     kPfProdQEmpty, kPfProdKEmpty, kPfMmaQFull, kPfMmaKFull, kPfMmaAccEmpty, kPfMmaTotal,
     kPfEpiAccFull, kPfEpiBufEmpty, kPfEpiTotal, kPfEpiTiles, kPfEpiMath, kPfSelBufFull,
-    kPfSelBusy, kPfSelTotal, kPfSelCut, kPfCvtK8Full, kPfCvtKEmpty, kPfCvtWork, kPfCvtTotal,
-    kPfSlots
+    kPfSelBusy, kPfSelTotal, kPfSelCut, kPfSplitWait, kPfSplitWork, kPfSplitTotal, kPfMmaIssue,
+    kPfMmaCommit, kPfSlots
 };
 #ifdef CSA_PROFILE
 constexpr int kProfCtas = 160;
@@ -140,15 +139,15 @@ struct Params {
     int nqb;      // query blocks per batch in this launch
     int nsplit;   // key-range splits per query block
     int n_items;
-    int stages;   // 16-bit key tiles in the MMA's ring
-    int stages8;  // E4M3 keys: raw tiles in the staging ring
+    int stages;   // key tiles in the MMA's ring (bf16, or E4M3 as stored)
     int cap;      // candidate list capacity per query and split
     int nmax;     // score-buffer keys per query (the longest item's key range)
-    int row_bytes;   // bytes of one swizzled operand row: min(128, 2*d)
+    int row_bytes;   // bytes of one swizzled bf16 operand row: min(128, 2*d)
     int n_chunks;    // d*2 / row_bytes
     // shared memory carve-up (byte offsets from the 1024-aligned base)
     int off_q, off_k, off_w, off_sel, off_bar, smem_bytes;
-    int off_k8;      // E4M3 keys: staging ring of raw key tiles
+    int off_e;       // E4M3 keys: the query block split into two E4M3 pieces
+    int off_sig;     // E4M3 keys: per-row query scales, two item halves
     const uint16_t *q; // only for L2 prefetch; loads go through the tensor map
     const float *w;
     const float *k_scale;
@@ -175,15 +174,17 @@ __device__ __forceinline__ int visible_count(const Params &p, long long t)
     return static_cast<int>(v > p.T ? p.T : v);
 }
 
-// Items run heaviest first: the last query blocks of a causal batch see the
-// most keys.
+// Items run heaviest first within a (batch, split): the last query blocks of
+// a causal batch see the most keys.  Query blocks vary fastest, so the CTAs
+// running at one time share a few sequences' key ranges and their key tiles
+// are read from HBM about once and then from L2.
 __device__ __forceinline__ Item decode_item(const Params &p, int id)
 {
     Item it;
-    it.split = id % p.nsplit;
-    const int r = id / p.nsplit;
-    it.b = r % p.B;
-    const int qbr = p.nqb - 1 - r / p.B;
+    const int qbr = p.nqb - 1 - id % p.nqb;
+    const int r = id / p.nqb;
+    it.split = r % p.nsplit;
+    it.b = r / p.nsplit;
     it.q0 = (p.qb_lo + qbr) * p.qps;
     it.nq = min(p.qps, p.S - it.q0);
     it.lrow = (it.b * p.nqb + qbr) * p.qps;
@@ -196,8 +197,9 @@ __device__ __forceinline__ Item decode_item(const Params &p, int id)
 
 struct Barriers {
     uint64_t q_full, q_empty, drain, q_ready;
+    uint64_t e_empty;                                     // E4M3: MMAs done with the pieces
+    uint64_t sig_full[2], sig_empty[2];                   // E4M3: row scales per item half
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
-    uint64_t k8_full[kMaxStages], k8_empty[kMaxStages];  // E4M3 staging ring
     uint64_t acc_full[2], acc_empty[2];
     uint64_t buf_full[2], buf_empty[2];                   // score-buffer halves
     uint32_t tmem_addr;
@@ -232,10 +234,12 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
                              uint8_t *smem, Barriers *bars, const WaitCtl &ctl)
 {
     int kload = 0, qload = 0;
+    int stage = 0, kphase = 0;   // ring position of the next key tile
     ProfAcc pa;
     Prof pf;
     const uint32_t q_bytes = static_cast<uint32_t>(p.N * p.d * 2);
-    const uint32_t k_bytes = static_cast<uint32_t>(kTileKeys * p.d * 2);
+    const int k_elem = p.key_fp8 ? 1 : 2;
+    const uint32_t k_bytes = static_cast<uint32_t>(kTileKeys * p.d * k_elem);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         pf.start();
@@ -267,38 +271,32 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
             const int row = it.b * p.T + t * kTileKeys;
             pf.start();
+            if (!wait_bounded(&bars->k_empty[stage], kphase ^ 1, ctl, kRoleProducer, id))
+                goto unwind;
+            pf.add(pa, kPfProdKEmpty, true);
+            mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
+            uint8_t *dst = smem + p.off_k + stage * k_bytes;
             if (p.key_fp8) {
-                // raw E4M3 tile (128 rows x d bytes) into the staging ring
-                const int stage = kload % p.stages8;
-                if (!wait_bounded(&bars->k8_empty[stage], ((kload / p.stages8) & 1) ^ 1, ctl,
-                                  kRoleProducer, id))
-                    goto unwind;
-                pf.add(pa, kPfProdKEmpty, true);
-                mbar_arrive_expect_tx(&bars->k8_full[stage], static_cast<uint32_t>(kTileKeys * p.d));
-                tma_load_2d(smem + p.off_k8 + stage * kTileKeys * p.d, tmK, &bars->k8_full[stage],
-                            0, row);
+                // E4M3 tile as stored: 128 rows of d bytes, swizzled at width d
+                tma_load_2d(dst, tmK, &bars->k_full[stage], 0, row);
             } else {
-                const int stage = kload % p.stages;
-                if (!wait_bounded(&bars->k_empty[stage], ((kload / p.stages) & 1) ^ 1, ctl,
-                                  kRoleProducer, id))
-                    goto unwind;
-                pf.add(pa, kPfProdKEmpty, true);
-                mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
-                uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
                 for (int c = 0; c < p.n_chunks; ++c)
                     tma_load_2d(dst + c * kTileKeys * p.row_bytes, tmK, &bars->k_full[stage],
                                 c * (p.row_bytes / 2), row);
             }
             ++kload;
+            if (++stage == p.stages) {
+                stage = 0;
+                kphase ^= 1;
+            }
         }
     }
 unwind:
     // Let every copy already issued land before the CTA can exit.
-    const int ring = p.key_fp8 ? p.stages8 : p.stages;
-    for (int s = 0; s < ring; ++s) {
+    for (int s = 0; s < p.stages; ++s) {
         if (kload > s) {
-            const int fills = (kload - s + ring - 1) / ring;
-            wait_drain(p.key_fp8 ? &bars->k8_full[s] : &bars->k_full[s], (fills - 1) & 1);
+            const int fills = (kload - s + p.stages - 1) / p.stages;
+            wait_drain(&bars->k_full[s], (fills - 1) & 1);
         }
     }
     if (qload > 0)
@@ -314,10 +312,13 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
     ProfAcc pa;
     Prof pf, pt;
     pt.start();
-    const uint32_t idesc = instr_desc_f16(p.N, p.key_fp8 ? 0 : 1); // f16 x f16 for E4M3 keys
+    // bf16 x bf16 (kind::f16), or E4M3 keys x E4M3 query pieces (kind::f8f6f4)
+    const uint32_t idesc = instr_desc_f16(p.N, p.key_fp8 ? 0 : 1);
     const int ksteps_per_chunk = p.row_bytes / 32;  // 16 elements (32 B) per MMA K step
     const uint32_t q_base = smem_u32(smem + p.off_q);
+    const uint32_t e_base = smem_u32(smem + p.off_e);
     const uint32_t k_base = smem_u32(smem + p.off_k);
+    const int k_tile_bytes = kTileKeys * p.d * (p.key_fp8 ? 1 : 2);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         pf.start();
@@ -337,26 +338,44 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
                 goto unwind;
             pf.add(pa, kPfMmaAccEmpty, true);
             tc_fence_after();
-            const uint32_t a_tile = k_base + stage * kTileKeys * p.d * 2;
+            const uint32_t a_tile = k_base + stage * k_tile_bytes;
             const uint32_t d_tmem = tmem_base + slot * kSlotCols;
-            for (int c = 0; c < p.n_chunks; ++c) {
-                for (int ks = 0; ks < ksteps_per_chunk; ++ks) {
-                    const uint64_t adesc = smem_desc_kmajor(
-                        a_tile + c * kTileKeys * p.row_bytes + ks * 32, p.row_bytes);
-                    const uint64_t bdesc =
-                        smem_desc_kmajor(q_base + c * p.N * p.row_bytes + ks * 32, p.row_bytes);
-                    mma_f16_ss(d_tmem, adesc, bdesc, idesc, (c | ks) != 0);
+            pf.start();
+            if (p.key_fp8) {
+                // 32 E4M3 per K step; the keys meet both query pieces, which
+                // sum in the one accumulator
+                for (int ks = 0; ks < p.d / 32; ++ks) {
+                    const uint64_t adesc = smem_desc_kmajor(a_tile + ks * 32, p.d);
+                    mma_f8_ss(d_tmem, adesc, smem_desc_kmajor(e_base + ks * 32, p.d), idesc,
+                              ks != 0);
+                    mma_f8_ss(d_tmem, adesc,
+                              smem_desc_kmajor(e_base + p.N * p.d + ks * 32, p.d), idesc, 1);
+                }
+            } else {
+                for (int c = 0; c < p.n_chunks; ++c) {
+                    for (int ks = 0; ks < ksteps_per_chunk; ++ks) {
+                        const uint64_t adesc = smem_desc_kmajor(
+                            a_tile + c * kTileKeys * p.row_bytes + ks * 32, p.row_bytes);
+                        const uint64_t bdesc = smem_desc_kmajor(
+                            q_base + c * p.N * p.row_bytes + ks * 32, p.row_bytes);
+                        mma_f16_ss(d_tmem, adesc, bdesc, idesc, (c | ks) != 0);
+                    }
                 }
             }
+            pf.add(pa, kPfMmaIssue, true);
+            pf.start();
             mma_commit(&bars->acc_full[slot]);
             mma_commit(&bars->k_empty[stage]);
+            pf.add(pa, kPfMmaCommit, true);
             ++acc_use;
             ++kuse;
         }
+        // the query operand's buffer is free once this item's MMAs are done
+        uint64_t *done = p.key_fp8 ? &bars->e_empty : &bars->q_empty;
         if (it.tile_end > it.tile_begin)
-            mma_commit(&bars->q_empty);
+            mma_commit(done);
         else
-            mbar_arrive(&bars->q_empty);
+            mbar_arrive(done);
         ++quse;
     }
 unwind:
@@ -366,141 +385,147 @@ unwind:
     pa.flush(true);
 }
 
-// ------------------------------------------------------------------ E4M3 converters
-// Byte offset of 16-byte unit `unit` of row r inside one swizzled operand
-// chunk (rows of row_bytes = 128 -> 128-byte swizzle, 64 -> 64-byte swizzle):
-// the unit index is XORed with row bits, as the TMA swizzle modes lay it out.
+// ------------------------------------------------------------------ query splitter (E4M3 keys)
+// Byte offset of 16-byte unit `unit` of row r in a swizzled operand block
+// whose rows are row_bytes (128, 64 or 32) long: the unit index is XORed with
+// row bits, as the TMA swizzle mode of that width lays it out.
 __device__ __forceinline__ uint32_t swizzled_unit(int r, int unit, int row_bytes)
 {
     const uint32_t o = static_cast<uint32_t>(r * row_bytes + unit * 16);
-    const uint32_t mask = row_bytes == 128 ? (7u << 7) : (3u << 7);
+    const uint32_t mask = row_bytes == 128 ? (7u << 7) : (row_bytes == 64 ? (3u << 7) : (1u << 7));
     return o ^ ((o & mask) >> 3);
 }
 
-// Four E4M3 values (one 32-bit word) -> four f16 (two words), exact.
-__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t b)
+// Two fp32 -> two E4M3, round to nearest even (|x| < 448 here); lo in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi)
 {
-    uint2 r;
-    asm("{\n\t.reg .b16 lo, hi;\n\t"
-        "mov.b32 {lo, hi}, %2;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}\n"
-        : "=r"(r.x), "=r"(r.y)
-        : "r"(b));
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
-// Two bf16 (one word) -> two f16 (one word), round to nearest.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w)
+// Two E4M3 (low byte first) -> two fp32, exact.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t b)
 {
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;"
-        : "=r"(r)
-        : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(__uint_as_float(w << 16)));
+    float2 r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t.reg .b32 h;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, %2;\n\t"
+        "mov.b32 {lo, hi}, h;\n\t"
+        "cvt.f32.f16 %0, lo;\n\t"
+        "cvt.f32.f16 %1, hi;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "h"(static_cast<unsigned short>(b)));
     return r;
 }
 
-constexpr int kConvThreads = 64;
-constexpr int kConvUnits = kTileKeys * 128 / 16 / kConvThreads; // 16-value units per thread (d <= 128)
+// Four bf16 (two words, element 0 in the low half of w0) times inv -> the two
+// E4M3 pieces: hi8 = E4M3(x), lo8 = E4M3(x - hi8), four bytes each.
+__device__ __forceinline__ void split4(uint32_t w0, uint32_t w1, float inv, uint32_t &hi8,
+                                       uint32_t &lo8)
+{
+    const float x0 = __uint_as_float(w0 << 16) * inv;
+    const float x1 = __uint_as_float(w0 & 0xFFFF0000u) * inv;
+    const float x2 = __uint_as_float(w1 << 16) * inv;
+    const float x3 = __uint_as_float(w1 & 0xFFFF0000u) * inv;
+    const uint32_t h01 = f32x2_to_e4m3x2(x0, x1);
+    const uint32_t h23 = f32x2_to_e4m3x2(x2, x3);
+    const float2 b01 = e4m3x2_to_f32x2(h01);
+    const float2 b23 = e4m3x2_to_f32x2(h23);
+    hi8 = h01 | (h23 << 16);
+    lo8 = f32x2_to_e4m3x2(x0 - b01.x, x1 - b01.y) | (f32x2_to_e4m3x2(x2 - b23.x, x3 - b23.y) << 16);
+}
 
-// Two warps (64 threads, `ct` = 0..63).  Per item: the query block, once the
-// TMA has landed it, from bf16 to f16 in place.  Per key tile: the staged
-// E4M3 tile to f16 in the swizzled key ring; a thread's units (and so its
-// source and destination offsets) are the same for every tile.  Each hand-off
-// fences the generic-proxy writes for the tensor cores, then one arrive per
-// warp.
-__device__ void run_converter(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl,
-                              int ct)
+// E4M3 keys: the tensor core multiplies E4M3 by E4M3, so warps 10-11 carry
+// each bf16 query row (one (query, head) pair) as sigma * (hi8 + lo8): sigma a
+// power of two that puts the row's largest |q| in [128, 256), hi8 the E4M3
+// rounding of q / sigma and lo8 the E4M3 rounding of what is left.  The
+// remainder has at most four significant bits, so the pair is exact whenever
+// it lies on E4M3's grid: for every element of at least 2^-9 of the row's
+// largest, and within 2^-17 of that largest otherwise (rows whose largest is
+// below 2^-100 take the scale of 2^-100).  hi8 and lo8 go to two
+// K-major operand blocks (rows of d bytes, swizzled at width d); sigma goes to
+// the epilogue, which folds it into the head weight (ReLU(sigma x) = sigma
+// ReLU(x) for sigma > 0).
+constexpr int kSplitThreads = 64;
+
+__device__ void run_qsplit(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl,
+                           int ct)
 {
     const int lane = ct & 31;
-    int kuse = 0, quse = 0;
-    const int units_q = p.N * p.d / 8;                 // 16-byte units of the query block
-    const int units_per_row = p.d / 16;                // 16 E4M3 values per unit
-    const int n_units = kTileKeys * units_per_row / kConvThreads;
-    const int elems_per_chunk_row = p.row_bytes / 2;
-    // Unit i of this thread is u = 64 i + ct: row 64 i / units_per_row + ct /
-    // units_per_row (a multiple of 8 rows apart for d <= 128, so the swizzle
-    // term is the same for every i) and the same columns for every i.
-    uint32_t dst_base[2];
-    {
-        const int r0 = ct / units_per_row;
-        const int j0 = (ct % units_per_row) * 16;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int j = j0 + 8 * half;
-            const int c = j / elems_per_chunk_row;
-            const int unit = (j % elems_per_chunk_row) / 8;
-            dst_base[half] =
-                static_cast<uint32_t>(c * kTileKeys * p.row_bytes) + swizzled_unit(r0, unit, p.row_bytes);
-        }
-    }
-    const uint32_t dst_step = static_cast<uint32_t>(kConvThreads / units_per_row * p.row_bytes);
+    const int units = p.row_bytes / 16;     // 8 bf16 per 16-byte unit, per chunk
+    const int eunits = p.d / 16;            // 16 E4M3 per 16-byte unit
+    const uint8_t *qs = smem + p.off_q;
+    uint8_t *e_hi = smem + p.off_e;
+    uint8_t *e_lo = e_hi + p.N * p.d;
+    int quse = 0;
     ProfAcc pa;
     Prof pf, pt;
     const bool rec = ct == 0;
     pt.start();
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
-        bool ok = wait_bounded(&bars->q_full, quse & 1, ctl, kRoleConvert, id);
+        const int par = quse & 1;
+        pf.start();
+        bool ok = wait_bounded(&bars->q_full, quse & 1, ctl, kRoleSplit, id);
+        // the MMAs of the previous item are done with the pieces, and the
+        // epilogue with this half's scales
+        ok = ok && wait_bounded(&bars->e_empty, (quse & 1) ^ 1, ctl, kRoleSplit, id);
+        ok = ok && wait_bounded(&bars->sig_empty[par], ((quse >> 1) & 1) ^ 1, ctl, kRoleSplit, id);
+        pf.add(pa, kPfSplitWait, rec);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok)
             return;
+        pf.start();
+        float *sig = reinterpret_cast<float *>(smem + p.off_sig) + par * p.N;
         if (it.tile_end > it.tile_begin) {
-            uint4 *qv = reinterpret_cast<uint4 *>(smem + p.off_q);
-            for (int u = ct; u < units_q; u += kConvThreads) {
-                uint4 x = qv[u];
-                x.x = bf16x2_to_f16x2(x.x);
-                x.y = bf16x2_to_f16x2(x.y);
-                x.z = bf16x2_to_f16x2(x.z);
-                x.w = bf16x2_to_f16x2(x.w);
-                qv[u] = x;
+            for (int r = ct; r < p.N; r += kSplitThreads) {
+                uint32_t m2 = 0;
+                for (int g = 0; g < p.d / 8; ++g) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(
+                        qs + (g / units) * p.N * p.row_bytes + swizzled_unit(r, g % units, p.row_bytes));
+                    m2 = __vmaxu2(m2, x.x & 0x7FFF7FFFu);
+                    m2 = __vmaxu2(m2, x.y & 0x7FFF7FFFu);
+                    m2 = __vmaxu2(m2, x.z & 0x7FFF7FFFu);
+                    m2 = __vmaxu2(m2, x.w & 0x7FFF7FFFu);
+                }
+                const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);   // bf16 bits of max |q|
+                int e = static_cast<int>((mb >> 7) & 0xFF) - 127;  // floor(log2 max |q|)
+                e = e < -100 ? -100 : (e > 127 ? 127 : e);
+                const float inv = __uint_as_float(static_cast<uint32_t>(7 - e + 127) << 23);
+                sig[r] = __uint_as_float(static_cast<uint32_t>(e - 7 + 127) << 23);
+                for (int v = 0; v < eunits; ++v) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int g = 2 * v + h;
+                        const uint4 x = *reinterpret_cast<const uint4 *>(
+                            qs + (g / units) * p.N * p.row_bytes + swizzled_unit(r, g % units, p.row_bytes));
+                        w[4 * h + 0] = x.x;
+                        w[4 * h + 1] = x.y;
+                        w[4 * h + 2] = x.z;
+                        w[4 * h + 3] = x.w;
+                    }
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        split4(w[2 * j], w[2 * j + 1], inv, hi[j], lo[j]);
+                    const uint32_t o = swizzled_unit(r, v, p.d);
+                    *reinterpret_cast<uint4 *>(e_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(e_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
             }
             fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&bars->q_ready);
-        ++quse;
-        for (int t = it.tile_begin; t < it.tile_end; ++t) {
-            const int stage = kuse % p.stages;      // slot in the f16 ring
-            const int stage8 = kuse % p.stages8;    // slot in the staging ring
-            pf.start();
-            ok = wait_bounded(&bars->k8_full[stage8], (kuse / p.stages8) & 1, ctl, kRoleConvert, id);
-            pf.add(pa, kPfCvtK8Full, rec);
-            pf.start();
-            ok = ok && wait_bounded(&bars->k_empty[stage], ((kuse / p.stages) & 1) ^ 1, ctl,
-                                    kRoleConvert, id);
-            pf.add(pa, kPfCvtKEmpty, rec);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok)
-                return;
-            pf.start();
-            const uint4 *src =
-                reinterpret_cast<const uint4 *>(smem + p.off_k8 + stage8 * kTileKeys * p.d);
-            uint8_t *dst = smem + p.off_k + stage * kTileKeys * p.d * 2;
-#pragma unroll
-            for (int i = 0; i < kConvUnits; ++i) {
-                if (i < n_units) {
-                    const uint4 x = src[i * kConvThreads + ct];
-                    const uint2 a = e4m3x4_to_f16x4(x.x);
-                    const uint2 b = e4m3x4_to_f16x4(x.y);
-                    const uint2 c = e4m3x4_to_f16x4(x.z);
-                    const uint2 d = e4m3x4_to_f16x4(x.w);
-                    *reinterpret_cast<uint4 *>(dst + dst_base[0] + i * dst_step) = make_uint4(a.x, a.y, b.x, b.y);
-                    *reinterpret_cast<uint4 *>(dst + dst_base[1] + i * dst_step) = make_uint4(c.x, c.y, d.x, d.y);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars->k_full[stage]);
-                mbar_arrive(&bars->k8_empty[stage8]);
-            }
-            pf.add(pa, kPfCvtWork, rec);
-            ++kuse;
+        if (lane == 0) {
+            mbar_arrive(&bars->q_empty);       // the bf16 block may be overwritten
+            mbar_arrive(&bars->q_ready);       // the pieces are in place
+            mbar_arrive(&bars->sig_full[par]); // and the scales
         }
+        pf.add(pa, kPfSplitWork, rec);
+        ++quse;
     }
-    pt.add(pa, kPfCvtTotal, rec);
+    pt.add(pa, kPfSplitTotal, rec);
     pa.flush(rec);
 }
 
@@ -531,6 +556,22 @@ __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int
             b = src[1];
         }
         wr[i] = make_float2(a, b);
+    }
+}
+
+// E4M3 keys: multiply the weights of fast_load_w by their rows' query scales.
+template <int FC, int FQ>
+__device__ __forceinline__ void fast_scale_w(const float *sig, int H, int j0, int lane,
+                                             float2 (&wr)[FC / 8])
+{
+    constexpr int RPQ = FC / 8 / FQ;
+#pragma unroll
+    for (int i = 0; i < FC / 8; ++i) {
+        const int j = j0 + i / RPQ;
+        const int h = 8 * (i % RPQ) + 2 * (lane & 3);
+        const float2 sg = *reinterpret_cast<const float2 *>(sig + j * H + h);
+        wr[i].x *= sg.x;
+        wr[i].y *= sg.y;
     }
 }
 
@@ -683,13 +724,23 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
         // (a group can run up to two items ahead of the other)
         float *w_s = reinterpret_cast<float *>(smem + p.off_w) +
                      ((p.tile_split ? wg : 0) * 2 + par) * p.qps * p.H;
+        // E4M3 keys: the splitter's per-row query scales of this item
+        const float *sig = reinterpret_cast<const float *>(smem + p.off_sig) + par * p.N;
+        bool oks = true;
+        if (p.key_fp8) {
+            pf.start();
+            oks = wait_bounded(&bars->sig_full[par], (it_count >> 1) & 1, ctl, kRoleEpilogue, id);
+            pf.add(pa, kPfEpiBufEmpty, rec);
+        }
         if constexpr (FC > 0) {
             fast_load_w<FC, FQ>(p, it, j0, lane, wr);
+            if (p.key_fp8 && oks)
+                fast_scale_w<FC, FQ>(sig, p.H, j0, lane, wr);
         } else {
             for (int r = 0; r < kWRegs; ++r) {
                 const int c = tid + r * kGroupThreads;
                 if (c < ncols)
-                    w_s[col0 + c] = wnext[r];
+                    w_s[col0 + c] = (p.key_fp8 && oks) ? wnext[r] * sig[col0 + c] : wnext[r];
             }
             const int nid = id + gridDim.x;
             if (nid < p.n_items) {
@@ -701,12 +752,17 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                 }
             }
         }
+        if (p.key_fp8) {
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars->sig_empty[par]);    // scales read
+        }
         // The selector must be done with this half (item it_count - 2).
         pf.start();
         const bool okw =
             wait_bounded(&bars->buf_empty[par], ((it_count >> 1) & 1) ^ 1, ctl, kRoleEpilogue, id);
         pf.add(pa, kPfEpiBufEmpty, rec);
-        ok = group_all(bar, kGroupThreads, ok && okw); // also publishes w_s
+        ok = group_all(bar, kGroupThreads, ok && okw && oks); // also publishes w_s
         if (!ok)
             break;
         float *buf = p.scores + (static_cast<size_t>(blockIdx.x) * 2 + par) * p.qps * p.nmax +
@@ -1099,16 +1155,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->q_empty, p.key_fp8 ? 2 : 1); // the splitter warps, or the MMA's commit
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->q_ready, 2);
+        mbar_init(&bars->e_empty, 1);
         for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&bars->k_full[s], p.key_fp8 ? 2 : 1); // converters, or the TMA's tx
+            mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
         }
-        for (int s = 0; s < p.stages8; ++s) {
-            mbar_init(&bars->k8_full[s], 1);
-            mbar_init(&bars->k8_empty[s], 2);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->sig_full[s], 2);
+            mbar_init(&bars->sig_empty[s], epi_warps);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->acc_full[s], 1);
@@ -1143,7 +1200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (warp == 9 && lane == 0)
             run_mma(p, smem, bars, tmem_base, ctl);
         else if (warp >= 10 && p.key_fp8)
-            run_converter(p, smem, bars, ctl, threadIdx.x - 320);
+            run_qsplit(p, smem, bars, ctl, threadIdx.x - 320);
     } else {
         regs_dec<kCtlRegs>();
         run_selector(p, smem, bars, ctl);

@@ -193,6 +193,19 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint
         : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f8f6f4 with the formats
+// the instruction descriptor names (E4M3 x E4M3 here), fp32 accumulate.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
@@ -273,19 +286,22 @@ __device__ __forceinline__ void reg_fence(uint32_t &r)
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor for a K-major operand tile whose rows are
-// `row_bytes` (128 -> 128B swizzle, 64 -> 64B swizzle) and whose 8-row groups
-// are 8*row_bytes apart.  Tiles start on 1024-byte boundaries; stepping K by 16
-// elements inside a swizzle row adds 32 bytes to the start address.
+// `row_bytes` (128, 64 or 32 -> the swizzle of that width) and whose 8-row
+// groups are 8*row_bytes apart.  Tiles start on 1024-byte boundaries; stepping
+// K by 32 bytes (16 bf16 or 32 E4M3 elements) inside a swizzle row adds 32
+// bytes to the start address.
 __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, int row_bytes)
 {
-    const uint64_t layout = row_bytes == 128 ? 2ull : 4ull; // SWIZZLE_128B : SWIZZLE_64B
+    // SWIZZLE_128B : SWIZZLE_64B : SWIZZLE_32B
+    const uint64_t layout = row_bytes == 128 ? 2ull : (row_bytes == 64 ? 4ull : 6ull);
     const uint64_t sbo = static_cast<uint64_t>(8 * row_bytes) >> 4;
     return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (sbo << 32) |
            (1ull << 46) | (layout << 61);
 }
 
 // Instruction descriptor: D fp32, A and B both bf16 (ab_bf16=1) or both f16,
-// both K-major, M = 128, N = n.
+// both K-major, M = 128, N = n.  With ab_bf16=0 the same bits select E4M3 x
+// E4M3 for kind::f8f6f4 (format code 0 in both kinds).
 __host__ __device__ constexpr uint32_t instr_desc_f16(int n, int ab_bf16)
 {
     return (1u << 4) | (static_cast<uint32_t>(ab_bf16) << 7) |
