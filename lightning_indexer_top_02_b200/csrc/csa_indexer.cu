@@ -258,7 +258,16 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
         }
     }
     const int tiles_max = max_tiles(a, p.q_offset);
-    const int min_split = (tiles_max * csa::kTileKeys + csa::kMaxItemKeys - 1) / csa::kMaxItemKeys;
+    // Longer key ranges split into items of at most max_item keys, so that an
+    // item's score buffer (qps x keys fp32, two per CTA) is re-read by the
+    // selector from L2 rather than HBM.  Each split adds a candidate list per
+    // query for the select kernel, which costs little when there are few query
+    // rows (decode): then items stop at 16,384 keys, else at kMaxItemKeys.
+    const long long rows_total = static_cast<long long>(p.B) * p.S;
+    int max_item = rows_total <= 16384 ? 16384 : csa::kMaxItemKeys;
+    if ((tiles_max * csa::kTileKeys + max_item - 1) / max_item > csa::kSelMaxSplits)
+        max_item = csa::kMaxItemKeys;
+    const int min_split = (tiles_max * csa::kTileKeys + max_item - 1) / max_item;
     if (nsplit < min_split)
         nsplit = min_split;
     if (nsplit < 1 || nsplit > csa::kSelMaxSplits)

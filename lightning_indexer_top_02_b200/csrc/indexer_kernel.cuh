@@ -855,6 +855,7 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
 constexpr int kSelPer = 16;
 constexpr int kSelChunk = kGroupThreads * kSelPer;   // 2048 scores
 constexpr int kSelShift = 21;                         // 2048 buckets
+constexpr int kSelShift2 = kSelShift - 11;            // second level inside one bucket
 
 struct SelectorScratch {
     GroupSmall gs;
@@ -1086,12 +1087,36 @@ __device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint
     int bd[4];
     sel_boundary(sc->hist, p.topk, &sc->gs, tid, bd);
     uint64_t lo;
-    if (bd[3] <= p.cap)
+    if (bd[3] <= p.cap) {
         lo = lo_key;                                   // every candidate fits
-    else if (bd[1] + bd[2] <= p.cap)
+    } else if (bd[1] + bd[2] <= p.cap) {
         lo = static_cast<uint64_t>(static_cast<uint32_t>(bd[0]) << kSelShift) << 32;
-    else
-        lo = sel_radix(sj, n, key0, lo_ord, p.topk, sc, tid);
+    } else {
+        // The boundary bucket (a quarter binade) holds too many keys: one
+        // more pass histograms its keys by the next 11 bits of the order image.
+        const uint32_t b1 = static_cast<uint32_t>(bd[0]);
+        const int above1 = bd[1];
+        for (int i = tid; i < kNbSelect; i += kGroupThreads)
+            sc->hist[i] = 0;
+        named_bar_sync(kBarSelect, kGroupThreads);
+        for (int base = 0; base < n; base += kSelChunk) {
+            uint32_t o[kSelPer];
+            sel_load(sj, base, n, tid, o);
+#pragma unroll
+            for (int e = 0; e < kSelPer; ++e)
+                if (sel_index(base, e, tid) < n && o[e] >= lo_ord && (o[e] >> kSelShift) == b1)
+                    atomicAdd(&sc->hist[(o[e] >> kSelShift2) & (kNbSelect - 1)], 1u);
+        }
+        named_bar_sync(kBarSelect, kGroupThreads);
+        int bd2[4];
+        sel_boundary(sc->hist, p.topk - above1, &sc->gs, tid, bd2);
+        if (above1 + bd2[1] + bd2[2] <= p.cap)
+            lo = static_cast<uint64_t>((b1 << kSelShift) |
+                                       (static_cast<uint32_t>(bd2[0]) << kSelShift2))
+                 << 32;
+        else
+            lo = sel_radix(sj, n, key0, lo_ord, p.topk, sc, tid);  // near-ties
+    }
     pf.add(pa, kPfSelCut, rec);
     return sel_emit(sj, n, key0, lo > lo_key ? lo : lo_key, list, sc, tid);
 }

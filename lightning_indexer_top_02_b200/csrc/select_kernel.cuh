@@ -71,9 +71,13 @@ __device__ __forceinline__ void sel_prefetch_l2(const void *src, uint32_t bytes)
 // For rows whose lists hold more keys than fit in registers: one histogram
 // pass over the lists in global memory (buckets = top 11 bits of the score
 // image) finds the bucket of the k-th largest key; returns the key L such that
-// every key >= L is at or above that bucket, with *count keys >= L.
+// every key >= L is at or above that bucket, with *count keys >= L.  With
+// b1 >= 0 the pass histograms only the keys of top-level bucket b1, by the
+// next 11 bits, for the `need`-th largest of them; *count then counts keys of
+// bucket b1 at or above the cut and *above those in higher sub-buckets.
 __device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *row_lists,
-                                         SelSmem *sm, int tid, int *count)
+                                         SelSmem *sm, int tid, int *count, int *above_out,
+                                         int b1 = -1, int need = -1)
 {
     const int lane = tid & 31, wid = tid >> 5;
     for (int i = tid; i < kSelNb; i += kSelThreads)
@@ -82,8 +86,13 @@ __device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *ro
     for (int s = 0; s < sp.nsplit; ++s) {
         const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
         const int n = sm->split_off[s + 1] - sm->split_off[s];
-        for (int j = tid; j < n; j += kSelThreads)
-            atomicAdd(&sm->hist[key_ord(src[j]) >> 21], 1u);
+        for (int j = tid; j < n; j += kSelThreads) {
+            const uint32_t o = key_ord(src[j]);
+            if (b1 < 0)
+                atomicAdd(&sm->hist[o >> 21], 1u);
+            else if ((o >> 21) == static_cast<uint32_t>(b1))
+                atomicAdd(&sm->hist[(o >> 10) & (kSelNb - 1)], 1u);
+        }
     }
     __syncthreads();
     // bucket of the k-th largest, top bucket first
@@ -110,7 +119,7 @@ __device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *ro
     for (int w = 0; w < kSelThreads / 32; ++w)
         higher += w > wid ? sm->gs.warp_sums[w] : 0u;
     const uint32_t above_thread = suf - sum + higher;
-    const uint32_t nd = static_cast<uint32_t>(sp.topk);
+    const uint32_t nd = static_cast<uint32_t>(b1 < 0 ? sp.topk : need);
     if (above_thread < nd && nd <= above_thread + sum) {
         uint32_t above = above_thread;
 #pragma unroll
@@ -118,6 +127,7 @@ __device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *ro
             if (above + c[j] >= nd) {
                 sm->misc[0] = tid * PER + j;
                 sm->misc[1] = static_cast<int>(above + c[j]);
+                sm->misc[3] = static_cast<int>(above);
                 break;
             }
             above += c[j];
@@ -125,7 +135,11 @@ __device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *ro
     }
     __syncthreads();
     *count = sm->misc[1];
-    const uint64_t L = static_cast<uint64_t>(static_cast<uint32_t>(sm->misc[0]) << 21) << 32;
+    *above_out = sm->misc[3];
+    const uint32_t cut = b1 < 0 ? static_cast<uint32_t>(sm->misc[0]) << 21
+                                : (static_cast<uint32_t>(b1) << 21) |
+                                      (static_cast<uint32_t>(sm->misc[0]) << 10);
+    const uint64_t L = static_cast<uint64_t>(cut) << 32;
     __syncthreads();
     return L;
 }
@@ -424,12 +438,23 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
         if (n_all > kSelKeys) {
             // keys at or above the histogram bucket of the k-th largest; an
             // exact radix cut when that bucket is too full
-            int kept_pre;
-            uint64_t L = sel_prefilter_global(sp, row_lists, sm, tid, &kept_pre);
-            if (kept_pre > kSelKeys)
-                L = sel_radix_global(sp, row_lists, sm, sp.topk, tid);
-            else
+            int kept_pre, above_pre;
+            uint64_t L = sel_prefilter_global(sp, row_lists, sm, tid, &kept_pre, &above_pre);
+            if (kept_pre > kSelKeys) {
+                // the boundary bucket is too full: split it by the next 11 bits
+                const int b1 = static_cast<int>(static_cast<uint32_t>(L >> 32) >> 21);
+                int kept2, above2;
+                const uint64_t L2 = sel_prefilter_global(sp, row_lists, sm, tid, &kept2, &above2,
+                                                         b1, sp.topk - above_pre);
+                if (above_pre + kept2 <= kSelKeys) {
+                    L = L2;
+                    n = above_pre + kept2;
+                } else {
+                    L = sel_radix_global(sp, row_lists, sm, sp.topk, tid);  // near-ties
+                }
+            } else {
                 n = kept_pre;
+            }
             if (tid == 0)
                 sm->misc[2] = 0;
             __syncthreads();

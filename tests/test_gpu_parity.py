@@ -236,6 +236,17 @@ def test_random_gate(lib):
     random_case(lib, wl, sample_rows(wl, 30), mode=1)
 
 
+def test_random_long_ranges(lib):
+    """Decode-sized batches over long key ranges (random normal): items of
+    about 15,000 keys whose k-th score often shares its quarter-binade histogram
+    bucket with more than the candidate list holds, so the selector refines
+    that bucket by a second histogram level; the select kernel merges three
+    lists per query through its (two-level) prefilter."""
+    wl = workloads.Workload("rlong", B=4, S=600, T=45000, H=64, d=128, m=4, topk=2048, seed=1900)
+    recalls = random_case(lib, wl, sample_rows(wl, 24, seed=19))
+    assert min(recalls) >= 0.999
+
+
 @pytest.mark.slow
 def test_dsa_prefill_full_size(lib):
     """DSA-style uncompressed prefill at its full size, sampled queries."""
