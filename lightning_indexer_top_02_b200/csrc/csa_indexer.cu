@@ -184,6 +184,8 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     p.tile_split = qps == 1 ? 1 : 0;
     if (p.tile_split)
         p.n_wg = 2;
+    // Small N: several key tiles share one accumulator slot, side by side.
+    p.tpg = csa::kSlotCols / p.N < csa::kMaxTpg ? csa::kSlotCols / p.N : csa::kMaxTpg;
 
     // Candidate list per (query, split): the top k plus room for the
     // selector's histogram bucket around the k-th score.

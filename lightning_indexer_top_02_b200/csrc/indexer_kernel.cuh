@@ -65,6 +65,7 @@ static_assert(2 * 128 * kEpiRegs + 2 * 128 * kCtlRegs == kThreads * kLaunchRegs,
 constexpr int kGroupThreads = 128;
 constexpr int kBarWg0 = 1, kBarWg1 = 2, kBarSelect = 3;  // named barriers
 constexpr int kMaxStages = 12;
+constexpr int kMaxTpg = 4;        // key tiles sharing one accumulator slot (small N)
 constexpr int kMaxTopk = 2048;
 constexpr int kNbSelect = 2048;  // buckets of the selector's histogram
 constexpr int kMaxItemKeys = 65536; // keys of one work item (longer ranges are split)
@@ -135,6 +136,7 @@ struct Params {
     int n_wg;     // epilogue warpgroups in use (1 or 2)
     int qpw;      // queries per epilogue warpgroup = qps / n_wg (or qps when tile_split)
     int tile_split; // one query per item: both warpgroups take every column, alternate tiles
+    int tpg;        // key tiles per accumulator slot (slot columns / N, at most kMaxTpg)
     int qb_lo;    // first query block (per batch) of this launch
     int nqb;      // query blocks per batch in this launch
     int nsplit;   // key-range splits per query block
@@ -326,20 +328,27 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
             goto unwind;
         pf.add(pa, kPfMmaQFull, true);
         tc_fence_after();
+        // Groups of up to tpg key tiles fill one accumulator slot side by side
+        // (N columns each), so that small N still hands the epilogue a full slot.
         for (int t = it.tile_begin; t < it.tile_end; ++t) {
+            const int g = (t - it.tile_begin) & (p.tpg - 1);     // place in the group
+            const bool last = g == p.tpg - 1 || t + 1 == it.tile_end;
+            const int slot = acc_use & 1;
+            if (g == 0) {
+                pf.start();
+                if (!wait_bounded(&bars->acc_empty[slot], ((acc_use >> 1) & 1) ^ 1, ctl, kRoleMma,
+                                  id))
+                    goto unwind;
+                pf.add(pa, kPfMmaAccEmpty, true);
+            }
             const int stage = kuse % p.stages;
             pf.start();
             if (!wait_bounded(&bars->k_full[stage], (kuse / p.stages) & 1, ctl, kRoleMma, id))
                 goto unwind;
             pf.add(pa, kPfMmaKFull, true);
-            const int slot = acc_use & 1;
-            pf.start();
-            if (!wait_bounded(&bars->acc_empty[slot], ((acc_use >> 1) & 1) ^ 1, ctl, kRoleMma, id))
-                goto unwind;
-            pf.add(pa, kPfMmaAccEmpty, true);
             tc_fence_after();
             const uint32_t a_tile = k_base + stage * k_tile_bytes;
-            const uint32_t d_tmem = tmem_base + slot * kSlotCols;
+            const uint32_t d_tmem = tmem_base + slot * kSlotCols + g * p.N;
             pf.start();
             if (p.key_fp8) {
                 // 32 E4M3 per K step; the keys meet both query pieces, which
@@ -364,10 +373,12 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
             }
             pf.add(pa, kPfMmaIssue, true);
             pf.start();
-            mma_commit(&bars->acc_full[slot]);
+            if (last) {
+                mma_commit(&bars->acc_full[slot]);
+                ++acc_use;
+            }
             mma_commit(&bars->k_empty[stage]);
             pf.add(pa, kPfMmaCommit, true);
-            ++acc_use;
             ++kuse;
         }
         // the query operand's buffer is free once this item's MMAs are done
@@ -606,7 +617,7 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0)
+    if (lane == 0 && acc_empty)
         mbar_arrive(acc_empty);
     float2 P[4][FQ];
 #pragma unroll
@@ -693,7 +704,7 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
         FC > 0 ? quarter * 32 + 16 * ((lane >> 1) & 1) + 8 * (lane & 1) + (lane >> 2)
                : quarter * 32 + lane;
     int acc_use = 0, it_count = 0;
-    int gtile = 0; // tiles of this CTA so far (tile_split: even ones are group 0's)
+    int gtile = 0; // tile groups of this CTA so far (tile_split: even ones are group 0's)
     ProfAcc pa;
     Prof pf, pt;
     const bool rec = wg == 0 && tid == 0;
@@ -768,33 +779,45 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
         float *buf = p.scores + (static_cast<size_t>(blockIdx.x) * 2 + par) * p.qps * p.nmax +
                      static_cast<size_t>(j0) * p.nmax;
 
+        int slot = 0;      // accumulator slot of the current tile group
+        bool mine = true;  // tile_split: the current group is this warpgroup's
         for (int t = it.tile_begin; t < it.tile_end && ok; ++t) {
-            if (p.tile_split && (gtile++ & 1) != wg)
-                continue;                            // the other group's tile
+            // tiles come in groups of tpg sharing one slot (as the MMA fills them)
+            const int g = (t - it.tile_begin) & (p.tpg - 1);
+            const bool last = g == p.tpg - 1 || t + 1 == it.tile_end;
+            if (g == 0) {
+                mine = !p.tile_split || (gtile++ & 1) == wg;
+                if (mine) {
+                    // tile_split: group w always drains slot w, every use flips its phase
+                    slot = p.tile_split ? wg : acc_use & 1;
+                    const uint32_t par = p.tile_split ? (acc_use & 1) : ((acc_use >> 1) & 1);
+                    pf.start();
+                    ok = wait_bounded(&bars->acc_full[slot], par, ctl, kRoleEpilogue, id);
+                    // the TMEM loads below are warp-collective: agree on the outcome first
+                    ok = __all_sync(0xffffffffu, ok);
+                    pf.add(pa, kPfEpiAccFull, rec);
+                    pf.count(pa, kPfEpiTiles, rec);
+                    ++acc_use;
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                }
+            }
+            if (!mine)
+                continue;                            // the other warpgroup's group
             const int s = t * kTileKeys + key_local;
             const size_t off = static_cast<size_t>(t - it.tile_begin) * kTileKeys + key_local;
             float kscale = 1.0f;
             if (p.key_fp8 && s < p.T)
                 kscale = p.k_scale[static_cast<size_t>(it.b) * p.T + s];
-            // tile_split: group w always drains slot w, every use flips its phase
-            const int slot = p.tile_split ? wg : acc_use & 1;
-            const uint32_t par = p.tile_split ? (acc_use & 1) : ((acc_use >> 1) & 1);
-            pf.start();
-            ok = wait_bounded(&bars->acc_full[slot], par, ctl, kRoleEpilogue, id);
-            // the TMEM loads below are warp-collective: agree on the outcome first
-            ok = __all_sync(0xffffffffu, ok);
-            pf.add(pa, kPfEpiAccFull, rec);
-            pf.count(pa, kPfEpiTiles, rec);
-            ++acc_use;
-            if (!ok)
-                break;
-            tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   slot * kSlotCols + col0;
+                                   slot * kSlotCols + g * p.N + col0;
             pf.start();
             if constexpr (FC > 0) {
                 float F[FQ];
-                fast_tile_scores<FC, FQ>(taddr, wr, &bars->acc_empty[slot], lane, F);
+                // the slot goes back to the MMA once its group's last tile is loaded
+                fast_tile_scores<FC, FQ>(taddr, wr, last ? &bars->acc_empty[slot] : nullptr, lane,
+                                         F);
 #pragma unroll
                 for (int q = 0; q < FQ; ++q)
                     buf[static_cast<size_t>(q) * p.nmax + off] = F[q] * kscale;
@@ -827,10 +850,12 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                         }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bars->acc_empty[slot]);
+                if (last) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->acc_empty[slot]);
+                }
             }
             pf.add(pa, kPfEpiMath, rec);
         }
