@@ -67,6 +67,24 @@ def test_fp8_scales_and_subnormals(lib):
     check_rows(inp, wl, gi, gs, rows, rtol=1e-5)
 
 
+def test_fp8_query_split_wide_range(lib):
+    """The tensor core takes each bf16 query row as sigma * (hi8 + lo8), two
+    E4M3 pieces.  Query elements spread over 18 binades put most of them on
+    the second piece (and some below E4M3's grid): the scores must still match
+    the exact fp64 scores to 2e-4 relative, which fails if lo8 were dropped or
+    mis-scaled (errors of order 2^-5 of each element)."""
+    wl = fp8(workloads.Workload("f8w", B=1, S=300, T=2500, H=64, d=128, m=1, topk=256, seed=1650))
+    inp = workloads.make_inputs(wl)
+    g = torch.Generator().manual_seed(1651)
+    shape = inp["q"].shape
+    mag = torch.pow(2.0, torch.empty(shape).uniform_(-14.0, 4.0, generator=g))
+    sign = torch.where(torch.rand(shape, generator=g) < 0.5, -1.0, 1.0)
+    inp["q"] = (sign * mag).to(torch.bfloat16)
+    gi, gs = run_gpu(lib, inp, wl)
+    rows = np.arange(0, wl.S, 7, dtype=np.int64)
+    check_rows(inp, wl, gi, gs, rows, rtol=2e-4)
+
+
 def check_rows(inp, wl, gi, gs, rows, *, mode=0, rtol):
     q, w, k, ks = workloads.as_numpy_bits(inp)
     ri, _, _, rc = oracle.topk(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
