@@ -30,6 +30,12 @@
  * q, k, k_scale and the outputs must be 16-byte aligned.  Inputs must be
  * finite; NaN or Inf inputs give unspecified (but memory-safe) results.
  *
+ * Arithmetic: products q.k accumulate in fp32 on the tensor cores, the head
+ * sum in fp32.  With E4M3 keys the key bytes are multiplied as stored and each
+ * query row (one (query, head) pair) is carried as sigma * (hi8 + lo8), two
+ * E4M3 pieces with a power-of-two sigma: exact for every element of at least
+ * 2^-9 of the row's largest |q|, within 2^-17 of that largest otherwise.
+ *
  * Supported shapes: H_I a power of two in [1, 256]; d in {32, 64, 128};
  * 1 <= topk <= 2048; m >= 1; T, S < 2^31.  Anything else returns
  * CSA_ERR_UNSUPPORTED before any launch.  There is no CPU fallback.
@@ -83,7 +89,7 @@ typedef struct {
 } csa_args_t;
 
 /*
- * The spec entry point: bf16 q and k, ReLU top-k, default q_offset.
+ * The plain entry point: bf16 q and k, ReLU top-k, default q_offset.
  * Needs scratch memory, which it takes with cudaMallocAsync on `stream` and
  * returns with cudaFreeAsync on the same stream (stream-ordered; no sync).
  */

@@ -110,7 +110,7 @@ def test_all_scores_tied(lib):
     check_exact(gi.reshape(-1, wl.topk), gs.reshape(-1, wl.topk), ri, rs, label="ties")
 
 
-def test_north_star_signature(lib):
+def test_plain_entry_point(lib):
     """csa_indexer_topk (bf16, ReLU top-k, default offset) through raw pointers."""
     wl = workloads.CONFIGS["tiny"]
     inp = workloads.make_inputs(wl)
