@@ -242,8 +242,39 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
     const uint32_t q_bytes = static_cast<uint32_t>(p.N * p.d * 2);
     const int k_elem = p.key_fp8 ? 1 : 2;
     const uint32_t k_bytes = static_cast<uint32_t>(kTileKeys * p.d * k_elem);
+    // One key tile into the ring (waits for its slot).
+    auto load_tile = [&](const Item &it, int t, int id) -> bool {
+        const int row = it.b * p.T + t * kTileKeys;
+        pf.start();
+        if (!wait_bounded(&bars->k_empty[stage], kphase ^ 1, ctl, kRoleProducer, id))
+            return false;
+        pf.add(pa, kPfProdKEmpty, true);
+        mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
+        uint8_t *dst = smem + p.off_k + stage * k_bytes;
+        if (p.key_fp8) {
+            // E4M3 tile as stored: 128 rows of d bytes, swizzled at width d
+            tma_load_2d(dst, tmK, &bars->k_full[stage], 0, row);
+        } else {
+            for (int c = 0; c < p.n_chunks; ++c)
+                tma_load_2d(dst + c * kTileKeys * p.row_bytes, tmK, &bars->k_full[stage],
+                            c * (p.row_bytes / 2), row);
+        }
+        ++kload;
+        if (++stage == p.stages) {
+            stage = 0;
+            kphase ^= 1;
+        }
+        return true;
+    };
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
+        // The item's first key tiles go into the ring as slots free up, before
+        // the query block, which waits for the previous item's MMAs: at the
+        // item boundary only the query block's latency is left exposed.
+        const int pre = min(it.tile_end - it.tile_begin, p.stages);
+        for (int t = it.tile_begin; t < it.tile_begin + pre; ++t)
+            if (!load_tile(it, t, id))
+                goto unwind;
         pf.start();
         if (!wait_bounded(&bars->q_empty, (qload & 1) ^ 1, ctl, kRoleProducer, id))
             goto unwind;
@@ -270,28 +301,9 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
                                 static_cast<uint32_t>(nx.nq * p.H * p.d * 2));
             }
         }
-        for (int t = it.tile_begin; t < it.tile_end; ++t) {
-            const int row = it.b * p.T + t * kTileKeys;
-            pf.start();
-            if (!wait_bounded(&bars->k_empty[stage], kphase ^ 1, ctl, kRoleProducer, id))
+        for (int t = it.tile_begin + pre; t < it.tile_end; ++t)
+            if (!load_tile(it, t, id))
                 goto unwind;
-            pf.add(pa, kPfProdKEmpty, true);
-            mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
-            uint8_t *dst = smem + p.off_k + stage * k_bytes;
-            if (p.key_fp8) {
-                // E4M3 tile as stored: 128 rows of d bytes, swizzled at width d
-                tma_load_2d(dst, tmK, &bars->k_full[stage], 0, row);
-            } else {
-                for (int c = 0; c < p.n_chunks; ++c)
-                    tma_load_2d(dst + c * kTileKeys * p.row_bytes, tmK, &bars->k_full[stage],
-                                c * (p.row_bytes / 2), row);
-            }
-            ++kload;
-            if (++stage == p.stages) {
-                stage = 0;
-                kphase ^= 1;
-            }
-        }
     }
 unwind:
     // Let every copy already issued land before the CTA can exit.
