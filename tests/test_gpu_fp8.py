@@ -49,6 +49,13 @@ def test_fp8_decode_splits_bit_exact(lib):
     exact_case(lib, fp8(wl))
 
 
+def test_fp8_single_query_bit_exact(lib):
+    """One query per sequence and 64 heads (N = 64): both epilogue warpgroups
+    take alternate groups of key tiles that share an accumulator slot."""
+    wl = workloads.Workload("f8one", B=5, S=1, T=3000, H=64, d=128, m=4, topk=300, seed=1550)
+    exact_case(lib, fp8(wl))
+
+
 def test_fp8_scales_and_subnormals(lib):
     """Keys drawn from every finite E4M3 code (subnormals, zeros of both signs,
     the largest value) with scales spanning many binades: the GPU must decode
