@@ -322,7 +322,10 @@ unwind:
 __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t tmem_base,
                         const WaitCtl &ctl)
 {
-    int kuse = 0, quse = 0, acc_use = 0;
+    int quse = 0, acc_use = 0;
+    // Ring position of the next key tile, kept incrementally: this thread's
+    // instruction latency between two tiles' MMAs idles the tensor pipe.
+    int stage = 0, kphase = 0;
     ProfAcc pa;
     Prof pf, pt;
     pt.start();
@@ -353,9 +356,8 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
                     goto unwind;
                 pf.add(pa, kPfMmaAccEmpty, true);
             }
-            const int stage = kuse % p.stages;
             pf.start();
-            if (!wait_bounded(&bars->k_full[stage], (kuse / p.stages) & 1, ctl, kRoleMma, id))
+            if (!wait_bounded(&bars->k_full[stage], kphase, ctl, kRoleMma, id))
                 goto unwind;
             pf.add(pa, kPfMmaKFull, true);
             tc_fence_after();
@@ -391,7 +393,10 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
             }
             mma_commit(&bars->k_empty[stage]);
             pf.add(pa, kPfMmaCommit, true);
-            ++kuse;
+            if (++stage == p.stages) {
+                stage = 0;
+                kphase ^= 1;
+            }
         }
         // the query operand's buffer is free once this item's MMAs are done
         uint64_t *done = p.key_fp8 ? &bars->e_empty : &bars->q_empty;
