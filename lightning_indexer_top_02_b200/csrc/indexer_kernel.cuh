@@ -319,6 +319,11 @@ unwind:
 }
 
 // ------------------------------------------------------------------ MMA issuer
+// MS selects the issue loop: 1 = bf16 keys with d = 128, 2 = E4M3 keys with
+// d = 128 (both fully unrolled with constant operand offsets, since this one
+// thread's instruction latency between tiles idles the tensor pipe), 0 = any
+// other head dimension.
+template <int MS>
 __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t tmem_base,
                         const WaitCtl &ctl)
 {
@@ -336,6 +341,11 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
     const uint32_t e_base = smem_u32(smem + p.off_e);
     const uint32_t k_base = smem_u32(smem + p.off_k);
     const int k_tile_bytes = kTileKeys * p.d * (p.key_fp8 ? 1 : 2);
+    // Descriptors count 16-byte units: byte offsets inside an operand add >> 4.
+    const uint64_t a_desc0 = smem_desc_kmajor(k_base, 128);
+    const uint32_t a_stage = static_cast<uint32_t>(k_tile_bytes >> 4);
+    const uint64_t b_desc0 = smem_desc_kmajor(MS == 2 ? e_base : q_base, 128);
+    const uint32_t b_chunk = static_cast<uint32_t>((p.N * 128) >> 4);  // bf16: next 64 elements; E4M3: lo8 block
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
         pf.start();
@@ -364,7 +374,22 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
             const uint32_t a_tile = k_base + stage * k_tile_bytes;
             const uint32_t d_tmem = tmem_base + slot * kSlotCols + g * p.N;
             pf.start();
-            if (p.key_fp8) {
+            if constexpr (MS == 1) {
+                const uint64_t a = a_desc0 + stage * a_stage;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16_ss(d_tmem, a + (c * ((kTileKeys * 128) >> 4) + 2 * ks),
+                                   b_desc0 + (c * b_chunk + 2 * ks), idesc, (c | ks) != 0);
+            } else if constexpr (MS == 2) {
+                const uint64_t a = a_desc0 + stage * a_stage;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    mma_f8_ss(d_tmem, a + 2 * ks, b_desc0 + 2 * ks, idesc, ks != 0);
+                    mma_f8_ss(d_tmem, a + 2 * ks, b_desc0 + (b_chunk + 2 * ks), idesc, 1);
+                }
+            } else if (p.key_fp8) {
                 // 32 E4M3 per K step; the keys meet both query pieces, which
                 // sum in the one accumulator
                 for (int ks = 0; ks < p.d / 32; ++ks) {
@@ -1264,8 +1289,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_dec<kCtlRegs>();
         if (warp == 8 && lane == 0)
             run_producer(p, &tmQ, &tmK, smem, bars, ctl);
-        else if (warp == 9 && lane == 0)
-            run_mma(p, smem, bars, tmem_base, ctl);
+        else if (warp == 9 && lane == 0) {
+            if (p.d == 128)
+                p.key_fp8 ? run_mma<2>(p, smem, bars, tmem_base, ctl)
+                          : run_mma<1>(p, smem, bars, tmem_base, ctl);
+            else
+                run_mma<0>(p, smem, bars, tmem_base, ctl);
+        }
         else if (warp >= 10 && p.key_fp8)
             run_qsplit(p, smem, bars, ctl, threadIdx.x - 320);
     } else {
