@@ -591,9 +591,8 @@ template <> struct Ld16x256<128> {
     static __device__ __forceinline__ void ld(uint32_t a, uint32_t (&v)[64]) { tmem_ld_16x256b_x16(a, v); }
 };
 
-// This thread's head weights, halved (the fast path forms w * ReLU(x) as
-// (w/2) * x + (w/2) * |x|, exact for the halving), for a warpgroup that reads
-// FC columns holding FQ queries: weight 2i+e belongs to column 8i + 2(lane%4) + e.
+// This thread's head weights for a warpgroup that reads FC columns holding FQ
+// queries: weight 2i+e belongs to column 8i + 2(lane%4) + e.
 template <int FC, int FQ>
 __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int j0, int lane,
                                             float2 (&wr)[FC / 8])
@@ -609,7 +608,7 @@ __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int
             a = src[0];
             b = src[1];
         }
-        wr[i] = make_float2(0.5f * a, 0.5f * b);
+        wr[i] = make_float2(a, b);
     }
 }
 
@@ -629,21 +628,16 @@ __device__ __forceinline__ void fast_scale_w(const float *sig, int H, int j0, in
     }
 }
 
-__device__ __forceinline__ float2 pair(uint32_t a, uint32_t b)
+__device__ __forceinline__ float2 relu2(uint32_t a, uint32_t b)
 {
-    return make_float2(__uint_as_float(a), __uint_as_float(b));
-}
-
-__device__ __forceinline__ float2 abs2(float2 x)
-{
-    return make_float2(fabsf(x.x), fabsf(x.y));
+    return make_float2(fmaxf(__uint_as_float(a), 0.0f), fmaxf(__uint_as_float(b), 0.0f));
 }
 
 // Scores of FQ queries for one key per thread.  The warp's two 16-lane loads
 // cover its 32 keys; thread t holds columns 8i + 2(t%4) + {0,1} of keys
 // t/4 + {0, 8, 16, 24}.  After the loads land the accumulator slot is released
 // (one arrive per warp).  Each thread then forms per-key partial sums over its
-// columns (column pairs with two packed FMAs); the quad (threads sharing t/4)
+// columns (column pairs with one packed FMA); the quad (threads sharing t/4)
 // exchanges halves twice so that thread t ends with the complete scores of
 // key row 16*((t>>1)&1) + 8*(t&1) + t/4 of the warp's 32.
 template <int FC, int FQ>
@@ -678,13 +672,10 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
         const int j = i / RPQ;
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub) {
-            // w * ReLU(x) = (w/2) * x + (w/2) * |x|: two packed FMAs, no max
-            const float2 xa = pair(va[4 * i + 2 * sub], va[4 * i + 2 * sub + 1]);
-            const float2 xb = pair(vb[4 * i + 2 * sub], vb[4 * i + 2 * sub + 1]);
-            P[sub][j] = __ffma2_rn(xa, wr[i], P[sub][j]);
-            P[sub][j] = __ffma2_rn(abs2(xa), wr[i], P[sub][j]);
-            P[2 + sub][j] = __ffma2_rn(xb, wr[i], P[2 + sub][j]);
-            P[2 + sub][j] = __ffma2_rn(abs2(xb), wr[i], P[2 + sub][j]);
+            P[sub][j] = __ffma2_rn(relu2(va[4 * i + 2 * sub], va[4 * i + 2 * sub + 1]), wr[i],
+                                   P[sub][j]);
+            P[2 + sub][j] = __ffma2_rn(relu2(vb[4 * i + 2 * sub], vb[4 * i + 2 * sub + 1]), wr[i],
+                                       P[2 + sub][j]);
         }
     }
     const bool b1 = (lane >> 1) & 1;
