@@ -21,7 +21,7 @@ def fp8(wl):
     return wl.replace(key_fp8=True)
 
 
-@pytest.mark.parametrize("H", [4, 16, 32, 64, 128])
+@pytest.mark.parametrize("H", [1, 4, 16, 32, 64, 128, 256])
 def test_fp8_heads_bit_exact(lib, H):
     wl = workloads.Workload("f8h", B=2, S=300, T=700, H=H, d=128, m=2, topk=100, seed=1200 + H)
     exact_case(lib, fp8(wl))
