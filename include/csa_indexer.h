@@ -128,10 +128,11 @@ csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
  * the library holds until the process exits.  The caller still passes all
  * inputs and outputs.  The first call on each device looks up that array's
  * device address (cudaGetSymbolAddress); make that first call before any
- * stream capture.  The scratch holds the candidate lists of the queries in
- * flight (B * queries-per-block * splits lists of about 2*topk 8-byte keys per
- * block of queries); when all of them do not fit, the call runs as several
- * launch chunks of query blocks.  If one query block of every sequence already
+ * stream capture.  The scratch holds the kernels' per-CTA score buffers and
+ * the candidate lists of the queries in flight (B * queries-per-block * splits
+ * lists of topk + max(256, topk/4) 8-byte keys per block of queries); when all
+ * of them do not fit, the call runs as several launch chunks of query blocks
+ * (and fewer CTAs when the score buffers alone would not fit).  If one query block of every sequence already
  * needs more than the array (very large B * topk), it returns
  * CSA_ERR_WORKSPACE and launches nothing.  All calls share the one array and
  * nothing in it needs to start at
