@@ -132,13 +132,12 @@ csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
  * the candidate lists of the queries in flight (B * queries-per-block * splits
  * lists of topk + max(256, topk/4) 8-byte keys per block of queries); when all
  * of them do not fit, the call runs as several launch chunks of query blocks
- * (and fewer CTAs when the score buffers alone would not fit).  If one query block of every sequence already
- * needs more than the array (very large B * topk), it returns
- * CSA_ERR_WORKSPACE and launches nothing.  All calls share the one array and
- * nothing in it needs to start at
- * zero, but two calls that overlap on the GPU (different streams, or
- * different host threads) race on it and give undefined results: serialise
- * them.
+ * (and fewer CTAs when the score buffers alone would not fit).  If one query
+ * block of every sequence already needs more than the array (very large
+ * B * topk), it returns CSA_ERR_WORKSPACE and launches nothing.  All calls
+ * share the one array and nothing in it needs to start at zero, but two calls
+ * that overlap on the GPU (different streams, or different host threads) race
+ * on it and give undefined results: serialise them.
  */
 #define CSA_NOALLOC_SCRATCH_BYTES (64ull << 20)
 csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStream_t stream);
