@@ -19,12 +19,14 @@
 //
 // Warp roles (512 threads, four warpgroups):
 //   warps 0..3   epilogue warpgroup 0: the first half of the item's queries
-//   warps 4..7   epilogue warpgroup 1: the second half (idle when qps == 1)
+//   warps 4..7   epilogue warpgroup 1: the second half (with one query per
+//                item both warpgroups read every column of alternate tile groups)
 //   warp 8       TMA producer: the query block once per item (with an L2
 //                prefetch of the next item's), key tiles into a ring
 //   warp 9       TMEM owner and MMA issuer (one thread): per key tile, d/16
 //                tcgen05.mma kind::f16 (M = 128 keys, N = qps*H_I) into one
-//                of two 256-column TMEM accumulators; with E4M3 keys, 2*d/32
+//                of two 256-column TMEM accumulators (up to four tiles side by
+//                side when N <= 128); with E4M3 keys, 2*d/32
 //                kind::f8f6f4 MMAs (the key tile as stored, times the two
 //                E4M3 pieces of the query block, summed in one accumulator)
 //   warps 10,11  E4M3 keys only: query splitter.  Each item's bf16 query rows
@@ -1057,7 +1059,8 @@ __device__ void sel_boundary(const uint32_t *hist, int need, GroupSmall *gs, int
 
 // Exact cut: the largest 64-bit key L such that exactly `need` keys with score
 // image >= lo_ord are >= L (more than `need` such keys exist; keys distinct).
-// Only for degenerate score ranges (a histogram bucket too full to keep).
+// Only for near-ties: even the second histogram level's boundary bucket holds
+// too many keys to keep.
 __device__ uint64_t sel_radix(const float *sj, int n, int key0, uint32_t lo_ord, int need,
                               SelectorScratch *sc, int tid)
 {
@@ -1127,7 +1130,8 @@ __device__ uint64_t sel_radix(const float *sj, int n, int key0, uint32_t lo_ord,
 // One query of a finished item: its n visible scores (keys key0..key0+n-1)
 // become a list of at most cap keys holding its top k -- all of them when
 // they fit (gated mode: all positive ones), else the keys at or above the
-// histogram bucket of the k-th largest, else exactly the top k.
+// histogram bucket of the k-th largest, else at or above its sub-bucket one
+// level down, else exactly the top k.
 __device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint64_t *list,
                          SelectorScratch *sc, int tid, ProfAcc &pa, bool rec)
 {
