@@ -240,6 +240,8 @@ def main():
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (B, S, T, H, d, m, topk, seed, causal, "
                          "key_fp8, gated), e.g. for a reduced profiling shape; the workload name records it")
+    ap.add_argument("--clocks-csv", default="",
+                    help="keep the raw nvidia-smi clock samples of the timed region here")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -317,8 +319,12 @@ def main():
     if rank == 0:
         props = torch.cuda.get_device_properties(dev)
         gid = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        sampler = ClockSampler(gid, os.path.join(ROOT, "gpurun_out", "bench_clocks.csv"))
+        clocks_csv = args.clocks_csv
+        if not clocks_csv:
+            import tempfile
+            fd, clocks_csv = tempfile.mkstemp(prefix="bench_clocks_", suffix=".csv")
+            os.close(fd)
+        sampler = ClockSampler(gid, clocks_csv)
         sampler.start()
     if world > 1:
         dist.barrier()
