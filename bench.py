@@ -33,7 +33,10 @@ import numpy as np  # noqa: E402
 
 import workloads  # noqa: E402
 
-DEFAULT_CONFIG = "dsa_prefill"
+# The V4-Flash-shaped prefill (S=65,536 queries over T=16,384 compressed keys,
+# H_I=64, d=128, top-2048, bf16): the shape the >= 60 % tensor-peak target names,
+# in the arithmetic (bf16 x bf16) whose dense peak is the roofline.
+DEFAULT_CONFIG = "v4flash_prefill"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -77,6 +80,22 @@ def measured_traffic(config: str, sha: str):
     return None
 
 
+def measured_fp8_peak(kind: str):
+    """E4M3 x E4M3 dense GEMM TFLOP/s measured on this GPU model ("burst" or
+    "sustained"), from profiles/peaks_fp8.txt, or None."""
+    path = os.path.join(ROOT, "profiles", "peaks_fp8.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == "e4m3" \
+                        and parts[1] == kind:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """The largest of every rank's value (the job is as slow as its slowest
     rank); the value itself on a single process."""
@@ -88,6 +107,15 @@ def max_over_ranks(value: float, device=None) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def check_world(gpus: int, world: int):
+    """``--gpus N`` must match the process count the launcher started (one
+    process per GPU under torchrun); returns an error message, or None."""
+    if gpus != world:
+        return (f"--gpus {gpus} but {world} process(es) were launched: run one process per GPU, "
+                f"e.g. python -m torch.distributed.run --nproc-per-node {gpus} bench.py --gpus {gpus}")
+    return None
 
 
 def dist_env():
@@ -105,10 +133,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str, out_path: str):
+    def __init__(self, gpu_id: str, out_path: str, keep: bool = True):
         self.out_path = out_path
         self.proc = None
         self.gpu_id = gpu_id
+        self.keep = keep
 
     def start(self):
         try:
@@ -135,12 +164,13 @@ class ClockSampler:
         with open(self.out_path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
+                if len(parts) >= 9:
                     rows.append(parts)
-                except ValueError:
-                    pass
+        if not self.keep:
+            try:
+                os.unlink(self.out_path)
+            except OSError:
+                pass
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -221,6 +251,7 @@ def config_dict(wl):
             "m": wl.m, "topk": wl.topk, "causal": wl.causal,
             "keys": "e4m3+fp32 scale" if wl.key_fp8 else "bf16",
             "mode": "sigmoid-gate" if wl.gated else "relu-topk",
+            **({"query_pieces": wl.q_pieces} if wl.key_fp8 and wl.q_pieces else {}),
             "values": wl.values, "l2": "flushed between timed steps (256 MiB write)",
             "parallelism": "replicas"}
 
@@ -252,7 +283,7 @@ def main():
         for item in args.set:
             field, _, value = item.partition("=")
             if field not in ("B", "S", "T", "H", "d", "m", "topk", "seed", "causal", "key_fp8",
-                             "gated"):
+                             "gated", "q_pieces"):
                 raise SystemExit(f"--set: unknown field {field!r}")
             flag = field in ("causal", "key_fp8", "gated")
             kw[field] = (value.lower() in ("1", "true")) if flag else int(value)
@@ -267,6 +298,9 @@ def main():
     import lightning_indexer_top_02_b200 as L
 
     rank, world, local = dist_env()
+    err = check_world(args.gpus, world)
+    if err:
+        raise SystemExit(err)
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
@@ -284,7 +318,7 @@ def main():
     out_sc = torch.empty((wl.B, wl.S, wl.topk), dtype=torch.float32, device=dev)
     mode = 1 if wl.gated else 0
     a = L.make_args(q, w, k, k_scale=ks, m=wl.m, topk=wl.topk, causal=wl.causal, mode=mode,
-                    out_idx=out_idx, out_score=out_sc)
+                    query_pieces=wl.q_pieces, out_idx=out_idx, out_score=out_sc)
     plan = L.csa_indexer_plan(a)
     ws_bytes = plan.workspace_bytes
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
@@ -324,7 +358,7 @@ def main():
             import tempfile
             fd, clocks_csv = tempfile.mkstemp(prefix="bench_clocks_", suffix=".csv")
             os.close(fd)
-        sampler = ClockSampler(gid, clocks_csv)
+        sampler = ClockSampler(gid, clocks_csv, keep=bool(args.clocks_csv))
         sampler.start()
     if world > 1:
         dist.barrier()
@@ -377,7 +411,7 @@ def main():
                 dks = torch.empty_like(ks) if ks is not None else None
                 doi, dos = torch.empty_like(out_idx), torch.empty_like(out_sc)
             aj = L.make_args(dq, dw, dk, k_scale=dks, m=wl.m, topk=wl.topk, causal=wl.causal,
-                             mode=mode, out_idx=doi, out_score=dos)
+                             mode=mode, query_pieces=wl.q_pieces, out_idx=doi, out_score=dos)
             hidx = torch.empty(out_idx.shape, dtype=torch.int32).pin_memory()
             hsc = torch.empty(out_sc.shape, dtype=torch.float32).pin_memory()
             bufs.append((dq, dw, dk, dks, doi, dos, aj, hidx, hsc))
@@ -431,9 +465,38 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
+
+        # The same steps in series on one stream: upload, call, read-back, with
+        # nothing overlapped (the latency of one request through the C ABI).
+        dq, dw, dk, dks, doi, dos, aj, hidx, hsc = bufs[0]
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s0.record(stream)
+        for i in range(n_e2e):
+            dq.copy_(hq, non_blocking=True)
+            dw.copy_(hw, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            if hks is not None:
+                dks.copy_(hks, non_blocking=True)
+            st = L.csa_indexer_topk_ex(aj, wsptr, ws_bytes, sptr)
+            if st != L.CSA_OK:
+                raise L.CsaError(st, "csa_indexer_topk_ex")
+            hidx.copy_(doi, non_blocking=True)
+            hsc.copy_(dos, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        serial_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, dev)
         e2e = {"value": queries * world / (e_ms / 1000.0), "unit": "queries/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e_ms, "pipelined": "copies overlap the neighbouring steps"}
+               "ms_per_step": e_ms,
+               "pipelined": "each step's upload and read-back overlap the neighbouring steps' "
+                            "kernels on two copy streams (serving loop)",
+               "serial": {"value": queries * world / (serial_ms / 1000.0), "unit": "queries/s",
+                          "ms_per_step": serial_ms,
+                          "what": "upload, call and read-back of each step in series on one stream"}}
 
     if rank != 0:
         if world > 1:
@@ -446,13 +509,16 @@ def main():
     sustained = timed_s > 0.5
     peak = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
     peak_name = f"{peak_src} bf16 dense ({'sustained' if sustained else 'burst'})"
+    fp8_measured = None
     if wl.key_fp8 and peak:
         # E4M3 x E4M3 MMAs: the FP8 peak is the measured bf16 one times the
-        # nominal dense ratio (4.5 / 2.25 PFLOP/s).  The query rides as two
-        # E4M3 pieces, so the tensor cores execute twice the algorithmic flops.
+        # nominal dense ratio (4.5 / 2.25 PFLOP/s).  A directly measured E4M3
+        # GEMM figure (profiles/peaks_fp8.txt) is reported beside it.
         peak = 2.0 * peak
         peak_name += " x 2 (nominal FP8 / bf16 ratio)"
+        fp8_measured = measured_fp8_peak("sustained" if sustained else "burst")
     fused_avg = statistics.mean(fused_ms)
+    step_avg = statistics.mean([f + s_ for f, s_ in zip(fused_ms, select_ms)])
     k_tflops = flops / (fused_avg / 1000.0) / 1e12
     sha = kernel_sources_sha()
     alg_bytes = wl.input_bytes() + wl.output_bytes()
@@ -461,18 +527,27 @@ def main():
               "kernel": "indexer_topk_kernel (fused scoring + candidate cut)",
               "kernel_ms": fused_avg, "select_kernel_ms": statistics.mean(select_ms),
               "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
-              "tensor_flops_executed_per_launch": (2 if wl.key_fp8 else 1) * flops,
+              "tensor_flops_executed_per_launch": (2 if wl.key_fp8 and wl.q_pieces != 1 else 1) * flops,
+              "step_kernels_ms": step_avg,
               "sources_sha": sha}
     if flops / alg_bytes < ridge:
         # few queries per key (single-query decode): the key stream bounds it
         gbs = alg_bytes / (fused_avg / 1000.0) / 1e9
+        step_gbs = alg_bytes / (step_avg / 1000.0) / 1e9
         roofline = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth",
+                    "step_achieved": step_gbs, "step_frac": step_gbs / peaks["hbm_gbs"],
                     **common}
     else:
+        step_tflops = flops / (step_avg / 1000.0) / 1e12
         roofline = {"bound": "tensor", "achieved": k_tflops, "peak": peak, "unit": "TFLOP/s",
                     "frac": k_tflops / peak if peak else None, "peak_source": peak_name,
+                    "step_achieved": step_tflops,
+                    "step_frac": step_tflops / peak if peak else None,
                     **common}
+        if fp8_measured:
+            roofline["fp8_measured_peak"] = fp8_measured
+            roofline["frac_of_fp8_measured"] = k_tflops / fp8_measured
     cpu = None
     if not args.no_cpu_baseline:
         cpu_inputs = inputs_for_oracle(wl, {"q": q, "w": w, "k": k, "k_scale": ks})
@@ -483,7 +558,8 @@ def main():
         "metric": "indexer queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 keys x e4m3 query pieces, fp32 accumulate" if wl.key_fp8 else "bf16",
+        "dtype": ("e4m3 keys x one e4m3 query piece, fp32 accumulate" if wl.q_pieces == 1 else
+                  "e4m3 keys x e4m3 query pieces, fp32 accumulate") if wl.key_fp8 else "bf16",
         "data": "synthetic", "config": config_dict(wl), "tflops": tflops,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * plan.launches,

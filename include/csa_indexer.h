@@ -27,8 +27,9 @@
  *   k_scale   [B, T]          float32, > 0 (CSA_KEY_E4M3 only)
  *   out_idx   [B, S, topk]    int32, key indices in [0, T) or -1
  *   out_score [B, S, topk]    float32
- * q, k, k_scale and the outputs must be 16-byte aligned.  Inputs must be
- * finite; NaN or Inf inputs give unspecified (but memory-safe) results.
+ * q and k must be 16-byte aligned (the tensor-memory copies read them);
+ * w, k_scale, out_idx and out_score 4-byte aligned.  Inputs must be finite;
+ * NaN or Inf inputs give unspecified (but memory-safe) results.
  *
  * Arithmetic: products q.k accumulate in fp32 on the tensor cores, the head
  * sum in fp32.  With E4M3 keys the key bytes are multiplied as stored and each
@@ -64,7 +65,10 @@ typedef enum {
     CSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes listed above       */
     CSA_ERR_WORKSPACE = 3,   /* caller workspace smaller than csa_indexer_workspace_size  */
     CSA_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, allocation, ...)      */
-    CSA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see csa_last_device_error) */
+    CSA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (see csa_last_device_error) */
+    CSA_ERR_DEBUG_CHECK = 6  /* debug build (-DCSA_DEBUG) only: a kernel's shared-memory,
+                                tensor-memory, buffer or output index failed its bounds
+                                check; the access was skipped (csa_last_device_error) */
 } csa_status_t;
 
 typedef enum { CSA_KEY_BF16 = 0, CSA_KEY_E4M3 = 1 } csa_key_dtype_t;
@@ -86,6 +90,14 @@ typedef struct {
     int num_splits;        /* key-range splits per query block; 0 = automatic  */
     int32_t *out_idx;      /* [B,S,topk]                                       */
     float *out_score;      /* [B,S,topk]                                       */
+    int query_pieces;      /* E4M3 keys only: how each bf16 query row meets the
+                              E4M3 keys on the tensor core.  0 or 2 (default):
+                              as sigma*(hi8 + lo8), two E4M3 pieces (exact for
+                              every element of at least 2^-9 of the row's
+                              largest |q|).  1: as sigma*hi8, one E4M3 rounding
+                              per element (relative error up to 2^-4): half the
+                              tensor work, at a cost in recall.  Must be 0 with
+                              bf16 keys.                                         */
 } csa_args_t;
 
 /*
@@ -124,8 +136,9 @@ csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
  * own pool.  The paper has no counterpart; this is a deployment variant.
  *
  * The call allocates nothing.  Its scratch is one fixed 64 MiB device array
- * inside this library (CSA_NOALLOC_SCRATCH_BYTES), which every GPU that loads
- * the library holds until the process exits.  The caller still passes all
+ * inside this library (CSA_NOALLOC_SCRATCH_BYTES); a GPU holds it from the
+ * library's first use on that device (at the latest the first call of this
+ * entry point there) until the process exits.  The caller still passes all
  * inputs and outputs.  The first call on each device looks up that array's
  * device address (cudaGetSymbolAddress); make that first call before any
  * stream capture.  The scratch holds the kernels' per-CTA score buffers and
@@ -170,8 +183,9 @@ const char *csa_status_string(csa_status_t status);
 
 /*
  * Synchronises `stream`, then reports (and clears) the device error word that
- * bounded waits set when they run out on the current device:
- * CSA_OK, CSA_ERR_TIMEOUT, or CSA_ERR_CUDA if the synchronisation failed.
+ * bounded waits set when they run out on the current device, and that the
+ * debug build's index checks set when one fails: CSA_OK, CSA_ERR_TIMEOUT,
+ * CSA_ERR_DEBUG_CHECK, or CSA_ERR_CUDA if the synchronisation failed.
  */
 csa_status_t csa_last_device_error(cudaStream_t stream);
 

@@ -18,7 +18,11 @@ import ctypes
 import os
 from typing import Optional
 
-from .build import LIB as LIB_PATH
+from .build import LIB as _BUILT_LIB
+
+# The library this binding loads: the in-tree build, or another build of the
+# same sources named by CSA_INDEXER_LIB (e.g. the -DCSA_DEBUG build).
+LIB_PATH = os.environ.get("CSA_INDEXER_LIB") or _BUILT_LIB
 
 CSA_OK = 0
 CSA_ERR_INVALID_ARG = 1
@@ -26,6 +30,7 @@ CSA_ERR_UNSUPPORTED = 2
 CSA_ERR_WORKSPACE = 3
 CSA_ERR_CUDA = 4
 CSA_ERR_TIMEOUT = 5
+CSA_ERR_DEBUG_CHECK = 6
 CSA_KEY_BF16 = 0
 CSA_KEY_E4M3 = 1
 CSA_MODE_TOPK = 0
@@ -52,6 +57,7 @@ class CsaArgs(ctypes.Structure):
         ("causal", ctypes.c_int), ("key_dtype", ctypes.c_int), ("mode", ctypes.c_int),
         ("q_offset", ctypes.c_longlong), ("num_splits", ctypes.c_int),
         ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
+        ("query_pieces", ctypes.c_int),
     ]
 
 
@@ -172,7 +178,7 @@ def _ptr(t):
 
 def make_args(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
               mode: int = CSA_MODE_TOPK, q_offset: int = -1, num_splits: int = 0,
-              out_idx=None, out_score=None) -> CsaArgs:
+              query_pieces: int = 0, out_idx=None, out_score=None) -> CsaArgs:
     """Pack torch tensors into the C argument struct (shapes read from q and k)."""
     import torch
 
@@ -188,6 +194,7 @@ def make_args(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
     a.mode = int(mode)
     a.q_offset = int(q_offset)
     a.num_splits = int(num_splits)
+    a.query_pieces = int(query_pieces)
     a.out_idx = out_idx.data_ptr() if out_idx is not None else None
     a.out_score = out_score.data_ptr() if out_score is not None else None
     return a
@@ -195,7 +202,8 @@ def make_args(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
 
 def indexer_topk(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
                  mode: int = CSA_MODE_TOPK, q_offset: int = -1, num_splits: int = 0,
-                 out_idx=None, out_score=None, workspace=None, stream=None):
+                 query_pieces: int = 0, out_idx=None, out_score=None, workspace=None,
+                 stream=None):
     """Run the indexer top-k on CUDA tensors; returns (out_idx, out_score).
 
     q: bf16 [B,S,H_I,d]; w: fp32 [B,S,H_I]; k: bf16 [B,T,d] or E4M3 bytes
@@ -215,8 +223,8 @@ def indexer_topk(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = Tru
     if out_score is None:
         out_score = torch.empty((B, S, topk), dtype=torch.float32, device=q.device)
     a = make_args(q, w, k, k_scale=k_scale, m=m, topk=topk, causal=causal, mode=mode,
-                  q_offset=q_offset, num_splits=num_splits, out_idx=out_idx,
-                  out_score=out_score)
+                  q_offset=q_offset, num_splits=num_splits, query_pieces=query_pieces,
+                  out_idx=out_idx, out_score=out_score)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ws_ptr, ws_bytes = None, 0

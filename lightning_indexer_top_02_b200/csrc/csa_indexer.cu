@@ -95,6 +95,9 @@ csa_status_t validate(const csa_args_t *a)
     if ((a->causal != 0 && a->causal != 1) || (a->mode != CSA_MODE_TOPK && a->mode != CSA_MODE_GATE) ||
         (a->key_dtype != CSA_KEY_BF16 && a->key_dtype != CSA_KEY_E4M3))
         return CSA_ERR_INVALID_ARG;
+    if (a->query_pieces < 0 || a->query_pieces > 2 ||
+        (a->key_dtype == CSA_KEY_BF16 && a->query_pieces != 0))
+        return CSA_ERR_INVALID_ARG;
     if (static_cast<long long>(a->B) * a->S == 0)
         return CSA_OK;
     if (!a->q || !a->w || !a->out_idx || !a->out_score)
@@ -159,6 +162,7 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     p.causal = a->causal;
     p.mode = a->mode;
     p.key_fp8 = a->key_dtype == CSA_KEY_E4M3;
+    p.q_pieces = p.key_fp8 ? (a->query_pieces == 1 ? 1 : 2) : 0;
     p.q_offset = a->q_offset >= 0 ? a->q_offset
                                   : (static_cast<long long>(a->T) * a->m > a->S
                                          ? static_cast<long long>(a->T) * a->m - a->S
@@ -204,7 +208,7 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     off += p.N * p.d * 2;
     if (p.key_fp8) {
         p.off_e = off;
-        off += 2 * p.N * p.d;
+        off += p.q_pieces * p.N * p.d;
     }
     p.off_k = off;
     const int w_bytes = 4 * p.qps * p.H * 4;           // w: per item parity (and group)
@@ -567,6 +571,7 @@ csa_status_t csa_indexer_topk(const void *q, const float *w, const void *k, int 
     a.mode = CSA_MODE_TOPK;
     a.q_offset = -1;
     a.num_splits = 0;
+    a.query_pieces = 0;
     a.out_idx = out_idx;
     a.out_score = out_score;
     return csa_indexer_topk_ex(&a, nullptr, 0, stream);
@@ -581,6 +586,7 @@ const char *csa_status_string(csa_status_t status)
     case CSA_ERR_WORKSPACE: return "workspace too small";
     case CSA_ERR_CUDA: return "CUDA runtime error";
     case CSA_ERR_TIMEOUT: return "device-side wait timed out";
+    case CSA_ERR_DEBUG_CHECK: return "debug-build index check failed on the device";
     }
     return "unknown status";
 }
@@ -597,7 +603,9 @@ csa_status_t csa_last_device_error(cudaStream_t stream)
     const int zero[4] = {0, 0, 0, 0};
     if (cudaMemcpyToSymbol(csa::g_csa_error, zero, sizeof zero) != cudaSuccess)
         return CSA_ERR_CUDA;
-    return h[0] == csa::kErrTimeout ? CSA_ERR_TIMEOUT : CSA_ERR_CUDA;
+    if (h[0] == csa::kErrTimeout)
+        return CSA_ERR_TIMEOUT;
+    return h[0] == csa::kErrDebugCheck ? CSA_ERR_DEBUG_CHECK : CSA_ERR_CUDA;
 }
 
 void csa_set_wait_limit(unsigned long long cycles)

@@ -132,6 +132,7 @@ struct Prof {
 
 struct Params {
     int B, S, T, H, d, m, topk, causal, mode, key_fp8;
+    int q_pieces;   // E4M3 keys: query pieces per (query, head) row (2: exact split, 1: one E4M3 rounding)
     long long q_offset;
     int qps;      // queries per item
     int N;        // MMA N = qps * H (<= 256)
@@ -251,6 +252,10 @@ __device__ void run_producer(const Params &p, const CUtensorMap *tmQ, const CUte
         if (!wait_bounded(&bars->k_empty[stage], kphase ^ 1, ctl, kRoleProducer, id))
             return false;
         pf.add(pa, kPfProdKEmpty, true);
+        if (!CSA_CHECK_INDEX(kChkKeyStage, stage, p.stages)) {
+            mbar_arrive(&bars->k_full[stage]);     // debug build: skip the copy, never hang
+            return true;
+        }
         mbar_arrive_expect_tx(&bars->k_full[stage], k_bytes);
         uint8_t *dst = smem + p.off_k + stage * k_bytes;
         if (p.key_fp8) {
@@ -346,7 +351,7 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
     // Descriptors count 16-byte units: byte offsets inside an operand add >> 4.
     const uint64_t a_desc0 = smem_desc_kmajor(k_base, 128);
     const uint32_t a_stage = static_cast<uint32_t>(k_tile_bytes >> 4);
-    const uint64_t b_desc0 = smem_desc_kmajor(MS == 2 ? e_base : q_base, 128);
+    const uint64_t b_desc0 = smem_desc_kmajor(MS >= 2 ? e_base : q_base, 128);
     const uint32_t b_chunk = static_cast<uint32_t>((p.N * 128) >> 4);  // bf16: next 64 elements; E4M3: lo8 block
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
         const Item it = decode_item(p, id);
@@ -376,7 +381,9 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
             const uint32_t a_tile = k_base + stage * k_tile_bytes;
             const uint32_t d_tmem = tmem_base + slot * kSlotCols + g * p.N;
             pf.start();
-            if constexpr (MS == 1) {
+            if (!CSA_CHECK_INDEX(kChkTmemMma, slot * kSlotCols + (g + 1) * p.N - 1, 2 * kSlotCols)) {
+                // debug build: a tile that would write past the allocation is skipped
+            } else if constexpr (MS == 1) {
                 const uint64_t a = a_desc0 + stage * a_stage;
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
@@ -391,15 +398,22 @@ __device__ void run_mma(const Params &p, uint8_t *smem, Barriers *bars, uint32_t
                     mma_f8_ss(d_tmem, a + 2 * ks, b_desc0 + 2 * ks, idesc, ks != 0);
                     mma_f8_ss(d_tmem, a + 2 * ks, b_desc0 + (b_chunk + 2 * ks), idesc, 1);
                 }
+            } else if constexpr (MS == 3) {
+                // one query piece: the key tile meets hi8 only
+                const uint64_t a = a_desc0 + stage * a_stage;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f8_ss(d_tmem, a + 2 * ks, b_desc0 + 2 * ks, idesc, ks != 0);
             } else if (p.key_fp8) {
-                // 32 E4M3 per K step; the keys meet both query pieces, which
+                // 32 E4M3 per K step; the keys meet every query piece, which
                 // sum in the one accumulator
                 for (int ks = 0; ks < p.d / 32; ++ks) {
                     const uint64_t adesc = smem_desc_kmajor(a_tile + ks * 32, p.d);
                     mma_f8_ss(d_tmem, adesc, smem_desc_kmajor(e_base + ks * 32, p.d), idesc,
                               ks != 0);
-                    mma_f8_ss(d_tmem, adesc,
-                              smem_desc_kmajor(e_base + p.N * p.d + ks * 32, p.d), idesc, 1);
+                    if (p.q_pieces == 2)
+                        mma_f8_ss(d_tmem, adesc,
+                                  smem_desc_kmajor(e_base + p.N * p.d + ks * 32, p.d), idesc, 1);
                 }
             } else {
                 for (int c = 0; c < p.n_chunks; ++c) {
@@ -490,6 +504,17 @@ __device__ __forceinline__ void split4(uint32_t w0, uint32_t w1, float inv, uint
     lo8 = f32x2_to_e4m3x2(x0 - b01.x, x1 - b01.y) | (f32x2_to_e4m3x2(x2 - b23.x, x3 - b23.y) << 16);
 }
 
+// Four bf16 (two words) times inv, each rounded once to E4M3 (the one-piece
+// query): four bytes, element 0 in the low byte.
+__device__ __forceinline__ uint32_t round4(uint32_t w0, uint32_t w1, float inv)
+{
+    const float x0 = __uint_as_float(w0 << 16) * inv;
+    const float x1 = __uint_as_float(w0 & 0xFFFF0000u) * inv;
+    const float x2 = __uint_as_float(w1 << 16) * inv;
+    const float x3 = __uint_as_float(w1 & 0xFFFF0000u) * inv;
+    return f32x2_to_e4m3x2(x0, x1) | (f32x2_to_e4m3x2(x2, x3) << 16);
+}
+
 // E4M3 keys: the tensor core multiplies E4M3 by E4M3, so warps 10-11 carry
 // each bf16 query row (one (query, head) pair) as sigma * (hi8 + lo8): sigma a
 // power of two that puts the row's largest |q| in [128, 256), hi8 the E4M3
@@ -500,7 +525,9 @@ __device__ __forceinline__ void split4(uint32_t w0, uint32_t w1, float inv, uint
 // below 2^-100 take the scale of 2^-100).  hi8 and lo8 go to two
 // K-major operand blocks (rows of d bytes, swizzled at width d); sigma goes to
 // the epilogue, which folds it into the head weight (ReLU(sigma x) = sigma
-// ReLU(x) for sigma > 0).
+// ReLU(x) for sigma > 0).  With one piece (q_pieces == 1) only hi8 is formed
+// and multiplied: half the tensor work, each query element rounded once to
+// E4M3 (relative error up to 2^-4).
 constexpr int kSplitThreads = 64;
 
 __device__ void run_qsplit(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl,
@@ -561,12 +588,18 @@ __device__ void run_qsplit(const Params &p, uint8_t *smem, Barriers *bars, const
                         w[4 * h + 3] = x.w;
                     }
                     uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        split4(w[2 * j], w[2 * j + 1], inv, hi[j], lo[j]);
                     const uint32_t o = swizzled_unit(r, v, p.d);
+                    if (p.q_pieces == 2) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            split4(w[2 * j], w[2 * j + 1], inv, hi[j], lo[j]);
+                        *reinterpret_cast<uint4 *>(e_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            hi[j] = round4(w[2 * j], w[2 * j + 1], inv);
+                    }
                     *reinterpret_cast<uint4 *>(e_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4 *>(e_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 }
             }
             fence_proxy_async_smem();
@@ -856,6 +889,11 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                 kscale = p.k_scale[static_cast<size_t>(it.b) * p.T + s];
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    slot * kSlotCols + g * p.N + col0;
+            const bool in_tmem =
+                CSA_CHECK_INDEX(kChkTmemEpi, slot * kSlotCols + g * p.N + col0 + ncols - 1, 2 * kSlotCols);
+            const bool in_buf = CSA_CHECK_INDEX(kChkScoreBuf, off, p.nmax);
+            (void)in_tmem;
+            (void)in_buf;
             pf.start();
             if constexpr (FC > 0) {
                 float F[FQ];
@@ -864,7 +902,8 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
                                          F);
 #pragma unroll
                 for (int q = 0; q < FQ; ++q)
-                    buf[static_cast<size_t>(q) * p.nmax + off] = F[q] * kscale;
+                    if (in_buf)
+                        buf[static_cast<size_t>(q) * p.nmax + off] = F[q] * kscale;
             } else {
                 const float *wsub = w_s + col0;
                 float acc = 0.0f;
@@ -961,7 +1000,7 @@ __device__ __forceinline__ int sel_index(int base, int e, int tid)
 
 // Appends every key of sj[0..n) (key index key0 + i) that is >= lo to `list`
 // in arbitrary order; returns how many.  One shared atomic per warp and chunk.
-__device__ int sel_emit(const float *sj, int n, int key0, uint64_t lo, uint64_t *list,
+__device__ int sel_emit(const float *sj, int n, int key0, uint64_t lo, uint64_t *list, int cap,
                         SelectorScratch *sc, int tid)
 {
     const int lane = tid & 31;
@@ -994,8 +1033,11 @@ __device__ int sel_emit(const float *sj, int n, int key0, uint64_t lo, uint64_t 
         int pos = __shfl_sync(0xffffffffu, wbase, 0) + incl - mine;
 #pragma unroll
         for (int e = 0; e < kSelPer; ++e)
-            if (keep & (1u << e))
-                list[pos++] = make_key(o[e], static_cast<uint32_t>(key0 + sel_index(base, e, tid)));
+            if (keep & (1u << e)) {
+                if (CSA_CHECK_INDEX(kChkListPos, pos, cap))
+                    list[pos] = make_key(o[e], static_cast<uint32_t>(key0 + sel_index(base, e, tid)));
+                ++pos;
+            }
     }
     named_bar_sync(kBarSelect, kGroupThreads);
     const int c = sc->out_cnt;
@@ -1140,7 +1182,7 @@ __device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint
     if (n <= 0)
         return 0;
     if (n <= p.cap)
-        return sel_emit(sj, n, key0, lo_key, list, sc, tid);
+        return sel_emit(sj, n, key0, lo_key, list, p.cap, sc, tid);
     Prof pf;
     pf.start();
     for (int i = tid; i < kNbSelect; i += kGroupThreads)
@@ -1189,7 +1231,7 @@ __device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint
             lo = sel_radix(sj, n, key0, lo_ord, p.topk, sc, tid);  // near-ties
     }
     pf.add(pa, kPfSelCut, rec);
-    return sel_emit(sj, n, key0, lo > lo_key ? lo : lo_key, list, sc, tid);
+    return sel_emit(sj, n, key0, lo > lo_key ? lo : lo_key, list, p.cap, sc, tid);
 }
 
 __device__ void run_selector(const Params &p, uint8_t *smem, Barriers *bars, const WaitCtl &ctl)
@@ -1270,6 +1312,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->buf_empty[s], kGroupThreads / 32);
         }
         bars->abort = 0;
+#ifdef CSA_DEBUG
+        // debug build: the plan's shared-memory carve-up fits the allocation
+        const int q_end = p.off_q + p.N * p.d * 2;
+        const int k_end = p.off_k + p.stages * kTileKeys * p.d * (p.key_fp8 ? 1 : 2);
+        if (!CSA_CHECK_INDEX(kChkQueryBlock, q_end - 1, p.key_fp8 ? p.off_e : p.off_k) ||
+            !CSA_CHECK_INDEX(kChkKeyStage, k_end - 1, p.off_w))
+            bars->abort = 1;
+#endif
         fence_mbar_init();
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
@@ -1294,10 +1344,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == 8 && lane == 0)
             run_producer(p, &tmQ, &tmK, smem, bars, ctl);
         else if (warp == 9 && lane == 0) {
-            if (p.d == 128)
-                p.key_fp8 ? run_mma<2>(p, smem, bars, tmem_base, ctl)
-                          : run_mma<1>(p, smem, bars, tmem_base, ctl);
-            else
+            if (p.d == 128) {
+                if (!p.key_fp8)
+                    run_mma<1>(p, smem, bars, tmem_base, ctl);
+                else if (p.q_pieces == 2)
+                    run_mma<2>(p, smem, bars, tmem_base, ctl);
+                else
+                    run_mma<3>(p, smem, bars, tmem_base, ctl);
+            } else
                 run_mma<0>(p, smem, bars, tmem_base, ctl);
         }
         else if (warp >= 10 && p.key_fp8)

@@ -69,6 +69,12 @@ __device__ int g_csa_error[4];
 
 enum : int { kErrTimeout = 5 };
 
+} // namespace csa
+
+#include "debug_check.cuh"
+
+namespace csa {
+
 // Wait budgets (cycles) at or above this use suspending probes.
 constexpr long long kSuspendBudget = 1ll << 22;
 

@@ -333,8 +333,10 @@ __device__ void sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEpt], int n, 
         for (int i = 0; i < kSelEpt; ++i) {
             if (db[i] <= dstar) {
                 const uint32_t slot = atomicAdd(&sm->hist[db[i]], 1u);
-                sm->out[slot] = e[i];
-                sm->out_b[slot] = static_cast<uint16_t>(db[i]);
+                if (CSA_CHECK_INDEX(kChkSelOut, slot, kSelKeys)) {
+                    sm->out[slot] = e[i];
+                    sm->out_b[slot] = static_cast<uint16_t>(db[i]);
+                }
             }
         }
         __syncthreads();
@@ -377,7 +379,8 @@ __device__ void sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEpt], int n, 
     __syncthreads();
     bitonic_sort_desc<kSelThreads>(sm->out, P, 0, tid);
     for (int i = tid; i < kept; i += kSelThreads)
-        sel_store(oi, os, i, sm->out[i]);
+        if (CSA_CHECK_INDEX(kChkSelOut, i, P))
+            sel_store(oi, os, i, sm->out[i]);
 }
 
 constexpr int kSelCtasPerSm = 3;
@@ -422,10 +425,13 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
             if (lane + 32 < sp.nsplit)
                 sm->split_off[lane + 33] = tot0 + x1;
         } else if (tid == 32) {
-            // warm L2 with the next row's first list
+            // Warm L2 with the next row's first list.  Rows past the last
+            // query of a partial query block have no list (their count slots
+            // were never written), and a count is never trusted beyond cap.
             const int rn = r + gridDim.x;
-            if (rn < sp.rows) {
-                const int cn = sp.counts[static_cast<size_t>(rn) * sp.nsplit];
+            if (rn < sp.rows && sp.qb_lo * sp.qps + rn % per_b < sp.S) {
+                int cn = sp.counts[static_cast<size_t>(rn) * sp.nsplit];
+                cn = cn < 0 ? 0 : (cn > sp.cap ? sp.cap : cn);
                 const uint32_t bytes = static_cast<uint32_t>((cn * 8 + 15) & ~15);
                 if (bytes > 0)
                     sel_prefetch_l2(sp.lists + static_cast<size_t>(rn) * sp.nsplit * sp.cap, bytes);
@@ -463,8 +469,11 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
                 const int ns = sm->split_off[s + 1] - sm->split_off[s];
                 for (int j = tid; j < ns; j += kSelThreads) {
                     const uint64_t x = src[j];
-                    if (x >= L)
-                        sm->out[atomicAdd(&sm->misc[2], 1)] = x;
+                    if (x >= L) {
+                        const int slot = atomicAdd(&sm->misc[2], 1);
+                        if (CSA_CHECK_INDEX(kChkSelOut, slot, kSelKeys))
+                            sm->out[slot] = x;
+                    }
                 }
             }
             __syncthreads();

@@ -118,26 +118,117 @@ def test_fp8_random_gate(lib):
 
 @pytest.mark.slow
 def test_long_prefill_fp8_full_size(lib):
-    """Long prefill (S=262,144, T=65,536, E4M3 keys) at full size, sampled queries."""
+    """Long prefill (S=262,144, T=65,536, E4M3 keys) at full size, 256+ sampled queries."""
     wl = workloads.CONFIGS["long_prefill_fp8"]
-    random_case(lib, wl, sample_rows(wl, 6, seed=3), rtol=3e-2)
+    random_case(lib, wl, sample_rows(wl, 256, seed=3), rtol=3e-2)
 
 
 @pytest.mark.slow
 def test_long_prefill_fp8_gated_full_size(lib):
     wl = workloads.CONFIGS["long_prefill_fp8_gated"]
-    random_case(lib, wl, sample_rows(wl, 6, seed=4), mode=1, rtol=3e-2)
+    random_case(lib, wl, sample_rows(wl, 256, seed=4), mode=1, rtol=3e-2)
 
 
 @pytest.mark.slow
 def test_decode_fp8_full_size(lib):
-    """Batched decode (B=32 x 64 queries at T=131,072, E4M3 keys), sampled queries."""
+    """Batched decode (B=32 x 64 queries at T=131,072, E4M3 keys), 256+ sampled queries."""
     wl = workloads.CONFIGS["decode_fp8"]
-    random_case(lib, wl, sample_rows(wl, 8, seed=5), rtol=3e-2)
+    random_case(lib, wl, sample_rows(wl, 256, seed=5), rtol=3e-2)
 
 
 @pytest.mark.slow
 def test_decode1_fp8_full_size(lib):
-    """One query per sequence (B=32, T=131,072, E4M3 keys), sampled queries."""
+    """One query per sequence (B=32, T=131,072, E4M3 keys), every query."""
     wl = workloads.CONFIGS["decode1_fp8"]
-    random_case(lib, wl, sample_rows(wl, 4, seed=6), rtol=3e-2)
+    random_case(lib, wl, np.arange(wl.B * wl.S, dtype=np.int64), rtol=3e-2)
+
+
+# ---------------------------------------------------------------- one-piece E4M3 query
+# With query_pieces = 1 each bf16 query row meets the E4M3 keys as one E4M3
+# rounding sigma * hi8 (half the tensor work of the exact two-piece split).
+# Integer-valued queries are exact in one piece, so those cases stay bit-exact;
+# random-normal queries lose up to 2^-4 relative per element, which the
+# accuracy bars of the two-piece path do not allow for: the random test
+# measures and records recall and score error against the oracle's exact
+# scores and holds them to the looser bar this mode documents.
+
+def one_piece_case(L, wl, *, mode=0):
+    inp = workloads.make_inputs(wl.replace(values="integer"))
+    q = inp["q"].cuda()
+    w = inp["w"].cuda()
+    k = inp["k"].cuda()
+    ks = inp["k_scale"].cuda()
+    idx, sc = L.indexer_topk(q, w, k, k_scale=ks, m=wl.m, topk=wl.topk, causal=wl.causal,
+                             mode=mode, query_pieces=1)
+    torch.cuda.synchronize()
+    assert L.csa_last_device_error(None) == L.CSA_OK
+    from parity import check_exact
+
+    ri, rs, _, _ = run_oracle(inp, wl, mode=mode)
+    check_exact(idx.cpu().numpy().reshape(-1, wl.topk), sc.cpu().numpy().reshape(-1, wl.topk),
+                ri, rs, label=f"{wl.name} one-piece")
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_one_piece_query_integer_bit_exact(lib, d):
+    wl = workloads.Workload("f8p1", B=2, S=300, T=900, H=64, d=d, m=2, topk=120, seed=1800 + d,
+                            key_fp8=True)
+    one_piece_case(lib, wl)
+
+
+def test_one_piece_query_gate_and_splits_bit_exact(lib):
+    one_piece_case(lib, workloads.Workload("f8p1g", B=1, S=400, T=1500, H=64, d=128, m=4,
+                                           topk=200, seed=1810, key_fp8=True), mode=1)
+    one_piece_case(lib, workloads.Workload("f8p1s", B=3, S=2, T=20000, H=64, d=128, m=4,
+                                           topk=512, seed=1811, key_fp8=True))
+
+
+def one_piece_recall(L, wl, rows):
+    """Recall and worst score error of the one-piece query on random inputs,
+    per sampled row, against the oracle's exact fp64 scores."""
+    from test_gpu_parity import oracle_rows
+
+    inp = workloads.make_inputs(wl, device="cuda")
+    idx, sc = L.indexer_topk(inp["q"], inp["w"], inp["k"], k_scale=inp["k_scale"], m=wl.m,
+                             topk=wl.topk, causal=wl.causal, query_pieces=1)
+    torch.cuda.synchronize()
+    assert L.csa_last_device_error(None) == L.CSA_OK
+    q, w, k, ks = workloads.as_numpy_bits(inp)
+    ri, _, _, rc = oracle.topk(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
+                               topk=wl.topk, causal=wl.causal, rows=rows)
+    gi = idx.cpu().numpy().reshape(-1, wl.topk)
+    gs = sc.cpu().numpy().reshape(-1, wl.topk)
+    recalls, errs = [], []
+    for n, (row, (I, vis)) in enumerate(zip(rows, oracle_rows(q, w, k, ks, wl, rows))):
+        cnt = int(rc[n])
+        sel = gi[row][gi[row] >= 0]
+        assert len(sel) == cnt and len(np.unique(sel)) == cnt and np.all(vis[sel])
+        kth = abs(I[ri[n][cnt - 1]]) if cnt else 1.0
+        errs.append(float(np.max(np.abs(gs[row][:cnt] - I[sel]) / np.maximum(np.abs(I[sel]), kth)))
+                    if cnt else 0.0)
+        recalls.append(len(np.intersect1d(sel, ri[n][:cnt])) / cnt if cnt else 1.0)
+    return np.array(recalls), np.array(errs)
+
+
+@pytest.mark.slow
+def test_one_piece_query_recall_long_prefill(lib):
+    """The one-piece query on the long-prefill shape, 256+ sampled rows: the
+    bar of this mode is mean recall >= 0.9 and every returned score within
+    0.1 of its exact value (relative to the k-th score); the exact-split
+    default is the mode that meets recall >= 0.999."""
+    wl = workloads.CONFIGS["long_prefill_fp8"]
+    rows = sample_rows(wl, 256, seed=21)
+    rec, err = one_piece_recall(lib, wl, rows)
+    print(f"one-piece query, long_prefill_fp8: recall mean {rec.mean():.4f} min {rec.min():.4f}, "
+          f"score error max {err.max():.3g} over {len(rows)} rows")
+    assert rec.mean() >= 0.9 and err.max() <= 0.1
+
+
+@pytest.mark.slow
+def test_one_piece_query_recall_decode(lib):
+    wl = workloads.CONFIGS["decode_fp8"]
+    rows = sample_rows(wl, 256, seed=22)
+    rec, err = one_piece_recall(lib, wl, rows)
+    print(f"one-piece query, decode_fp8: recall mean {rec.mean():.4f} min {rec.min():.4f}, "
+          f"score error max {err.max():.3g} over {len(rows)} rows")
+    assert rec.mean() >= 0.9 and err.max() <= 0.1

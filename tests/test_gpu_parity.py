@@ -201,8 +201,24 @@ def test_wait_timeout_is_reported(lib):
 
 # ---------------------------------------------------------------- random-normal inputs
 
-def random_case(L, wl, rows, *, mode=0, rtol=1e-2):
-    inp = workloads.make_inputs(wl, device="cuda")
+def oracle_rows(q, w, k, ks, wl, rows):
+    """The oracle's fp64 scores and visibility of each sampled row, computed
+    on all host threads (the oracle's calls release the interpreter lock)."""
+    import concurrent.futures
+    import os
+
+    def one(row):
+        b, i = divmod(int(row), wl.S)
+        return oracle.score_row(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
+                                b=b, i=i, causal=wl.causal)
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        return list(ex.map(one, rows))
+
+
+def random_case(L, wl, rows, *, mode=0, rtol=1e-2, inp=None):
+    if inp is None:
+        inp = workloads.make_inputs(wl, device="cuda")
     gi, gs = run_gpu(L, inp, wl, mode=mode)
     q, w, k, ks = workloads.as_numpy_bits(inp)
     ri, _, _, rc = oracle.topk(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
@@ -210,20 +226,32 @@ def random_case(L, wl, rows, *, mode=0, rtol=1e-2):
     gi = gi.reshape(-1, wl.topk)
     gs = gs.reshape(-1, wl.topk)
     recalls = []
-    for n, row in enumerate(rows):
-        b, i = divmod(int(row), wl.S)
-        I, vis = oracle.score_row(q, w, k, ks, B=wl.B, S=wl.S, T=wl.T, H=wl.H, d=wl.d, m=wl.m,
-                                  b=b, i=i, causal=wl.causal)
+    for n, (row, (I, vis)) in enumerate(zip(rows, oracle_rows(q, w, k, ks, wl, rows))):
         recalls.append(check_random_row(gi[row], gs[row], ri[n], rc[n], I, vis, topk=wl.topk,
                                         gate=mode == 1, rtol=rtol, label=f"{wl.name} row {row}"))
     return recalls
 
 
-def sample_rows(wl, n, seed=0):
+def sample_rows(wl, n, seed=0, heavy=4):
+    """n random query rows, plus the first and last rows of the first and
+    last sequences and the last `heavy` rows of the last sequence (the
+    heaviest query block: the most visible keys)."""
     rng = np.random.default_rng(seed)
-    rows = np.unique(np.concatenate([rng.integers(0, wl.B * wl.S, n),
-                                     [0, wl.B * wl.S - 1, wl.S - 1]]))
+    last = wl.B * wl.S
+    rows = np.unique(np.concatenate([rng.integers(0, last, n),
+                                     [0, last - 1, wl.S - 1],
+                                     np.arange(max(0, last - heavy), last)]))
     return rows.astype(np.int64)
+
+
+def exact_sampled_case(L, wl, rows, *, mode=0):
+    """Integer-valued inputs at any size: the GPU's rows must equal the
+    oracle's bit for bit on the sampled rows."""
+    inp = workloads.make_inputs(wl.replace(values="integer"), device="cuda")
+    gi, gs = run_gpu(L, inp, wl, mode=mode)
+    ri, rs, _, _ = run_oracle(inp, wl, mode=mode, rows=rows)
+    check_exact(gi.reshape(-1, wl.topk)[rows], gs.reshape(-1, wl.topk)[rows], ri, rs,
+                label=f"{wl.name} (integer, {len(rows)} sampled rows)")
 
 
 def test_random_small_recall(lib):
@@ -249,13 +277,31 @@ def test_random_long_ranges(lib):
 
 @pytest.mark.slow
 def test_dsa_prefill_full_size(lib):
-    """DSA-style uncompressed prefill at its full size, sampled queries."""
+    """DSA-style uncompressed prefill at its full size, 256+ sampled queries."""
     wl = workloads.CONFIGS["dsa_prefill"]
-    random_case(lib, wl, sample_rows(wl, 24, seed=1))
+    random_case(lib, wl, sample_rows(wl, 256, seed=1))
 
 
 @pytest.mark.slow
 def test_v4flash_prefill_full_size(lib):
-    """V4-Flash-shaped prefill at its full size (S=65,536, T=16,384), sampled queries."""
+    """V4-Flash-shaped prefill at its full size (S=65,536, T=16,384), 256+ sampled queries."""
     wl = workloads.CONFIGS["v4flash_prefill"]
-    random_case(lib, wl, sample_rows(wl, 16, seed=2))
+    random_case(lib, wl, sample_rows(wl, 256, seed=2))
+
+
+@pytest.mark.slow
+def test_dsa_prefill_integer_full_size(lib):
+    """Integer-valued inputs at the full DSA prefill size (S=T=8192, top-2048):
+    every key of the 8192-key items goes through the selector's histogram
+    levels and near-tie cut with dense exact ties, and the GPU must match the
+    oracle bit for bit on 512+ sampled rows."""
+    wl = workloads.CONFIGS["dsa_prefill"]
+    exact_sampled_case(lib, wl, sample_rows(wl, 512, seed=11))
+
+
+@pytest.mark.slow
+def test_v4flash_prefill_integer_full_size(lib):
+    """Integer-valued inputs at the full V4-Flash prefill size (items of up
+    to 16,384 keys), bit for bit on 512+ sampled rows."""
+    wl = workloads.CONFIGS["v4flash_prefill"]
+    exact_sampled_case(lib, wl, sample_rows(wl, 512, seed=12))

@@ -59,3 +59,24 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
     with contextlib.redirect_stdout(buf):
         rc = bench.run_reference(Args(), bench.workloads.CONFIGS["tiny"])
     assert rc == 0 and buf.getvalue() == ""
+
+
+def test_gpus_must_match_launched_processes():
+    """``--gpus N`` with fewer (or more) processes than N is refused, so that
+    one process can never be reported as N GPUs."""
+    assert bench.check_world(1, 1) is None
+    assert bench.check_world(4, 4) is None
+    assert "torch.distributed.run" in bench.check_world(8, 1)
+    assert bench.check_world(2, 4) is not None
+
+
+def test_bench_refuses_gpus_without_launcher():
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--steps", "1"],
+                       capture_output=True, text=True, cwd=root, env=env)
+    assert r.returncode != 0
+    assert "--gpus 2 but 1 process" in r.stderr

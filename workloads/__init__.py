@@ -46,6 +46,7 @@ class Workload:
     key_fp8: bool = False
     gated: bool = False
     values: str = "normal"  # "normal" | "integer"
+    q_pieces: int = 0       # E4M3 keys: query pieces on the tensor core (0/2 exact split, 1 one rounding)
     seed: int = 0
     note: str = ""
 
