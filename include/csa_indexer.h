@@ -155,6 +155,64 @@ csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace,
 #define CSA_NOALLOC_SCRATCH_BYTES (64ull << 20)
 csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStream_t stream);
 
+/*
+ * Sparse attention over the selected keys: the step that consumes the
+ * indexer's output ("StreamIndex: Memory-Bounded Compressed Sparse Attention
+ * via Streaming Top-k", abstract: a sparse attention kernel reads only the
+ * selected compressed keys).  For every batch b, query row i and head g < HA:
+ *
+ *   J = idx[b,i,0..n), the selected keys, where n is the first slot that holds
+ *       no key in [0, T) (the indexer lists its selection first and pads with
+ *       -1; anything after the first such slot is ignored)
+ *   out[b,i,g,:] = sum_j softmax_j( scale * q[b,i,g,:] . k[b,J_j,:] ) * v[b,J_j,:]
+ *   (zeros when n = 0)
+ *
+ * One compressed cache row per key is shared by all heads.  Layouts (DEVICE
+ * memory owned by the caller, row-major):
+ *   q    [B, S, HA, Dk]  bfloat16, 16-byte aligned
+ *   k    [B, T, Dk]      bfloat16, 16-byte aligned
+ *   v    value row s of batch b at v + (b*T + s) * ld_v elements (bfloat16,
+ *        16-byte aligned, ld_v >= Dv and ld_v * 2 a multiple of 16); v = k
+ *        with ld_v = Dk reads the values as the first Dv elements of each key
+ *        row (a latent cache)
+ *   idx  [B, S, topk]    int32 (the indexer's out_idx)
+ *   out  [B, S, HA, Dv]  float32, 16-byte aligned
+ * Arithmetic: q.k on the tensor cores (bf16, fp32 accumulate), softmax in
+ * fp32 (exp2 domain), the probabilities rounded to bf16 for P.V (fp32
+ * accumulate).  Supported: 1 <= HA <= 128; Dk, Dv multiples of 64 up to 256.
+ * Stream-ordered; status codes as above; no allocation.
+ */
+typedef struct {
+    const void *q;
+    const void *k;
+    const void *v;
+    long long ld_v;
+    const int32_t *idx;
+    int B, S, T, HA, Dk, Dv, topk;
+    float scale;
+    float *out;
+} csa_attn_args_t;
+
+csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaStream_t stream);
+
+/*
+ * OR-union of several layers' selections ("FlashMemory-DeepSeek-V4:
+ * Lightning Index Ultra-Long Context via Lookahead Sparse Attention", "What
+ * carries the argument": the gated decisions of a few layers are combined by
+ * OR-union).  lists is a HOST array of n_lists (1..8) DEVICE pointers, each
+ * [rows, topk] int32 (an indexer's out_idx; entries outside [0, T) are
+ * padding).  For every row, out[row, 0..count) receives the distinct keys any
+ * list holds, in ascending key order, at most cap of them (the smallest keys
+ * when the union is larger; size cap = n_lists * topk to keep every key), and
+ * out[row, count..cap) is -1.  out [rows, cap] and count [rows] are device
+ * int32, 4-byte aligned.  T up to about 1.8 million keys (a bitmap of the
+ * row's keys in shared memory); larger returns CSA_ERR_UNSUPPORTED.
+ * Stream-ordered; no allocation.
+ */
+csa_status_t csa_union_selections(const int32_t *const *lists, int n_lists, int rows, int topk,
+                                  int T, int cap, int32_t *out, int32_t *count,
+                                  cudaStream_t stream);
+
 /* How csa_indexer_topk_ex would run a call (for benchmarks and tests). */
 typedef struct {
     int grid;              /* CTAs of the fused kernel (persistent, <= SM count) */

@@ -37,9 +37,10 @@ CSA_MODE_TOPK = 0
 CSA_MODE_GATE = 1
 
 EXPORTS = ("csa_indexer_topk", "csa_indexer_topk_ex", "csa_indexer_workspace_size",
-           "csa_indexer_plan", "csa_indexer_topk_noalloc", "csa_status_string",
-           "csa_last_device_error", "csa_set_wait_limit", "csa_set_launch_events",
-           "csa_version")
+           "csa_indexer_plan", "csa_indexer_topk_noalloc", "csa_sparse_attention",
+           "csa_union_selections",
+           "csa_status_string", "csa_last_device_error", "csa_set_wait_limit",
+           "csa_set_launch_events", "csa_version")
 
 
 class CsaError(RuntimeError):
@@ -58,6 +59,16 @@ class CsaArgs(ctypes.Structure):
         ("q_offset", ctypes.c_longlong), ("num_splits", ctypes.c_int),
         ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
         ("query_pieces", ctypes.c_int),
+    ]
+
+
+class CsaAttnArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("ld_v", ctypes.c_longlong), ("idx", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("S", ctypes.c_int), ("T", ctypes.c_int), ("HA", ctypes.c_int),
+        ("Dk", ctypes.c_int), ("Dv", ctypes.c_int), ("topk", ctypes.c_int),
+        ("scale", ctypes.c_float), ("out", ctypes.c_void_p),
     ]
 
 
@@ -92,6 +103,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.csa_indexer_workspace_size.restype = ctypes.c_size_t
     lib.csa_indexer_topk_noalloc.argtypes = [ctypes.POINTER(CsaArgs), P]
     lib.csa_indexer_topk_noalloc.restype = I
+    lib.csa_union_selections.argtypes = [P, I, I, I, I, I, P, P, P]
+    lib.csa_union_selections.restype = I
+    lib.csa_sparse_attention.argtypes = [ctypes.POINTER(CsaAttnArgs), P]
+    lib.csa_sparse_attention.restype = I
     lib.csa_indexer_plan.argtypes = [ctypes.POINTER(CsaArgs), ctypes.POINTER(CsaPlan)]
     lib.csa_indexer_plan.restype = I
     lib.csa_status_string.argtypes = [I]
@@ -128,6 +143,10 @@ def csa_indexer_workspace_size(args: CsaArgs) -> int:
 def csa_indexer_topk_noalloc(args: CsaArgs, stream_ptr) -> int:
     """The allocation-free entry point (fixed in-library scratch; see the header)."""
     return load_library().csa_indexer_topk_noalloc(ctypes.byref(args), stream_ptr)
+
+
+def csa_sparse_attention(args: CsaAttnArgs, stream_ptr) -> int:
+    return load_library().csa_sparse_attention(ctypes.byref(args), stream_ptr)
 
 
 def csa_indexer_plan(args: CsaArgs) -> CsaPlan:
@@ -234,3 +253,71 @@ def indexer_topk(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = Tru
     if st != CSA_OK:
         raise CsaError(st, "csa_indexer_topk_ex")
     return out_idx, out_score
+
+
+def sparse_attention(q, k, idx, *, scale: float, v=None, dv: Optional[int] = None, out=None,
+                     stream=None):
+    """Attention of every head over the keys ``idx`` selects, on CUDA tensors.
+
+    q: bf16 [B,S,HA,Dk]; k: bf16 [B,T,Dk]; idx: int32 [B,S,topk] (the
+    indexer's out_idx); v: bf16 [B,T,Dv], or None to read the values as the
+    first ``dv`` elements of each key row (one latent cache).  Returns out
+    fp32 [B,S,HA,Dv] (allocated if not given).
+    """
+    import torch
+
+    B, S, HA, Dk = q.shape
+    T = k.shape[1]
+    if v is None:
+        Dv = int(dv) if dv is not None else Dk
+        vt, ld_v = k, Dk
+    else:
+        Dv = v.shape[-1]
+        vt, ld_v = v, Dv
+    for name, t in (("q", q), ("k", k), ("v", vt), ("idx", idx)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if out is None:
+        out = torch.empty((B, S, HA, Dv), dtype=torch.float32, device=q.device)
+    a = CsaAttnArgs()
+    a.q, a.k, a.v, a.ld_v, a.idx = q.data_ptr(), k.data_ptr(), vt.data_ptr(), ld_v, idx.data_ptr()
+    a.B, a.S, a.T, a.HA, a.Dk, a.Dv, a.topk = B, S, T, HA, Dk, Dv, idx.shape[-1]
+    a.scale = float(scale)
+    a.out = out.data_ptr()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = csa_sparse_attention(a, ctypes.c_void_p(stream.cuda_stream))
+    if st != CSA_OK:
+        raise CsaError(st, "csa_sparse_attention")
+    return out
+
+
+def csa_union_selections(list_ptrs, rows: int, topk: int, T: int, cap: int, out_ptr, count_ptr,
+                         stream_ptr) -> int:
+    arr = (ctypes.c_void_p * len(list_ptrs))(*list_ptrs)
+    return load_library().csa_union_selections(arr, len(list_ptrs), rows, topk, T, cap, out_ptr,
+                                               count_ptr, stream_ptr)
+
+
+def union_selections(idx_lists, T: int, cap: Optional[int] = None, stream=None):
+    """OR-union per row of several [.., topk] int32 CUDA selections (same
+    shape); returns (keys [rows, cap] ascending with -1 padding, count [rows])."""
+    import torch
+
+    first = idx_lists[0]
+    topk = first.shape[-1]
+    rows = first.numel() // topk
+    for t in idx_lists:
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.int32 or t.shape != first.shape:
+            raise ValueError("selections must be contiguous int32 CUDA tensors of one shape")
+    cap = len(idx_lists) * topk if cap is None else int(cap)
+    out = torch.empty(first.shape[:-1] + (cap,), dtype=torch.int32, device=first.device)
+    count = torch.empty(first.shape[:-1], dtype=torch.int32, device=first.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(first.device)
+    st = csa_union_selections([t.data_ptr() for t in idx_lists], rows, topk, T, cap,
+                              ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(count.data_ptr()),
+                              ctypes.c_void_p(stream.cuda_stream))
+    if st != CSA_OK:
+        raise CsaError(st, "csa_union_selections")
+    return out, count

@@ -5,6 +5,7 @@
 // and then the exact top-k selection over its candidate lists.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdint>
 #include <cstdlib>
@@ -14,6 +15,8 @@
 #include "csa_indexer.h"
 #include "indexer_kernel.cuh"
 #include "select_kernel.cuh"
+#include "sparse_attn_kernel.cuh"
+#include "union_kernel.cuh"
 
 namespace {
 
@@ -24,6 +27,16 @@ constexpr int kSmemLimit = 232448; // 227 KB of dynamic shared memory per CTA on
 constexpr unsigned long long kDefaultWaitLimit = 4000000000ull;
 
 unsigned long long g_wait_limit = kDefaultWaitLimit;
+
+// NVTX range around a host-side region (a profiler's timeline shows each
+// call and each launch chunk by name; without a profiler attached the calls
+// are no-ops).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Measurement hook: events recorded around this thread's launches.
 thread_local cudaEvent_t *t_events = nullptr;
@@ -335,13 +348,15 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
 }
 
 bool make_tmap(CUtensorMap *tm, CUtensorMapDataType dt, const void *base, long long rows, int cols,
-               int box_cols, int box_rows, CUtensorMapSwizzle swz, int elem_bytes = 2)
+               int box_cols, int box_rows, CUtensorMapSwizzle swz, int elem_bytes = 2,
+               long long row_stride = 0)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
         return false;
     const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(row_stride > 0 ? row_stride : cols) *
+                                   elem_bytes};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estride[2] = {1, 1};
     return enc(tm, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
@@ -425,6 +440,7 @@ csa_status_t launch(const csa_args_t *a, const Plan &plan, void *ws, cudaStream_
     for (int qb_lo = 0; qb_lo < plan.nqb_total; qb_lo += plan.qb_chunk) {
         const int nqb = plan.nqb_total - qb_lo < plan.qb_chunk ? plan.nqb_total - qb_lo
                                                               : plan.qb_chunk;
+        NvtxRange chunk_range("csa launch chunk: fused scoring + exact select");
         p.qb_lo = qb_lo;
         p.nqb = nqb;
         p.n_items = p.B * nqb * p.nsplit;
@@ -515,6 +531,7 @@ csa_status_t csa_indexer_plan(const csa_args_t *args, csa_plan_t *out)
 csa_status_t csa_indexer_topk_ex(const csa_args_t *args, void *workspace, size_t workspace_bytes,
                                  cudaStream_t stream)
 {
+    NvtxRange range("csa_indexer_topk_ex");
     csa_status_t st = validate(args);
     if (st != CSA_OK)
         return st;
@@ -627,6 +644,162 @@ int csa_version(void) { return kVersion; }
 } // extern "C"
 
 // ---------------------------------------------------------------------------
+// Sparse attention over the selected keys.
+namespace {
+
+csa_status_t validate_attn(const csa_attn_args_t *a)
+{
+    if (!a)
+        return CSA_ERR_INVALID_ARG;
+    if (a->B < 0 || a->S < 0 || a->T < 0 || a->HA <= 0 || a->Dk <= 0 || a->Dv <= 0 ||
+        a->topk <= 0 || a->ld_v < a->Dv || !(a->scale == a->scale))
+        return CSA_ERR_INVALID_ARG;
+    if (static_cast<long long>(a->B) * a->S == 0)
+        return CSA_OK;
+    if (!a->q || !a->idx || !a->out || (a->T > 0 && (!a->k || !a->v)))
+        return CSA_ERR_INVALID_ARG;
+    if (!aligned(a->q, 16) || (a->k && !aligned(a->k, 16)) || (a->v && !aligned(a->v, 16)) ||
+        !aligned(a->idx, 4) || !aligned(a->out, 16) || (a->ld_v * 2) % 16 != 0)
+        return CSA_ERR_INVALID_ARG;
+    if (a->HA > csa::attn::kRows || a->Dk % 64 != 0 || a->Dk > 256 || a->Dv % 64 != 0 ||
+        a->Dv > 256)
+        return CSA_ERR_UNSUPPORTED;
+    const long long rows_q = static_cast<long long>(a->B) * a->S * a->HA;
+    if (rows_q + csa::attn::kRows >= (1ll << 31) || static_cast<long long>(a->B) * a->T >= (1ll << 31) ||
+        static_cast<long long>(a->B) * a->S * a->topk >= (1ll << 40))
+        return CSA_ERR_UNSUPPORTED;
+    return CSA_OK;
+}
+
+__global__ void zero_kernel(float *x, long long n)
+{
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        x[i] = 0.0f;
+}
+
+} // namespace
+
+extern "C" csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaStream_t stream)
+{
+    NvtxRange range("csa_sparse_attention");
+    const csa_status_t st = validate_attn(args);
+    if (st != CSA_OK)
+        return st;
+    const long long rows = static_cast<long long>(args->B) * args->S;
+    if (rows == 0)
+        return CSA_OK;
+    if (args->T == 0) {
+        zero_kernel<<<256, 256, 0, stream>>>(args->out, rows * args->HA * args->Dv);
+        return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+    }
+    using namespace csa::attn;
+    AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    p.B = args->B;
+    p.S = args->S;
+    p.T = args->T;
+    p.HA = args->HA;
+    p.Dk = args->Dk;
+    p.Dv = args->Dv;
+    p.topk = args->topk;
+    p.sl2 = args->scale * 1.4426950408889634f;
+    p.idx = args->idx;
+    p.out = args->out;
+    p.wait_limit = static_cast<long long>(g_wait_limit);
+    // shared memory: the query block, the key and value rings, P, barriers
+    p.k_stage_bytes = kKeys * p.Dk * 2;
+    p.v_stage_bytes = kKeys * p.Dv * 2;
+    const int q_bytes = kRows * p.Dk * 2;
+    const int p_bytes = kRows * kKeys * 2;
+    const int fixed = q_bytes + p_bytes + static_cast<int>(sizeof(AttnBarriers)) + 64 + 1024;
+    p.stages = fixed + kMaxStages * (p.k_stage_bytes + p.v_stage_bytes) <= kSmemLimit ? kMaxStages : 1;
+    if (fixed + p.stages * (p.k_stage_bytes + p.v_stage_bytes) > kSmemLimit)
+        return CSA_ERR_UNSUPPORTED;
+    p.off_q = 0;
+    p.off_k = q_bytes;
+    p.off_v = p.off_k + p.stages * p.k_stage_bytes;
+    p.off_p = p.off_v + p.stages * p.v_stage_bytes;
+    p.off_bar = p.off_p + p_bytes;
+    int smem_bytes = p.off_bar + static_cast<int>(sizeof(AttnBarriers)) + 64 + 1024;
+    // more than half of the SM: one CTA per SM, so its 512-column TMEM
+    // allocation never waits on a neighbour
+    if (smem_bytes < kSmemLimit / 2 + 1024)
+        smem_bytes = kSmemLimit / 2 + 1024;
+
+    CUtensorMap tmQ, tmK, tmV;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap(&tmQ, bf, args->q, rows * p.HA, p.Dk, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&tmK, bf, args->k, static_cast<long long>(p.B) * p.T, p.Dk, 64, 1,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&tmV, bf, args->v, static_cast<long long>(p.B) * p.T, p.Dv, 64, 1,
+                   CU_TENSOR_MAP_SWIZZLE_128B, 2, args->ld_v))
+        return CSA_ERR_CUDA;
+    if (cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    const int sms = device_sms();
+    if (sms <= 0)
+        return CSA_ERR_CUDA;
+    const int grid = rows < sms ? static_cast<int>(rows) : sms;
+    if (!mark(0, stream))
+        return CSA_ERR_CUDA;
+    sparse_attn_kernel<<<grid, kThreads, smem_bytes, stream>>>(tmQ, tmK, tmV, p);
+    if (cudaGetLastError() != cudaSuccess)
+        return CSA_ERR_CUDA;
+    if (!mark(1, stream))
+        return CSA_ERR_CUDA;
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// OR-union of several layers' selections.
+extern "C" csa_status_t csa_union_selections(const int32_t *const *lists, int n_lists, int rows,
+                                             int topk, int T, int cap, int32_t *out,
+                                             int32_t *count, cudaStream_t stream)
+{
+    NvtxRange range("csa_union_selections");
+    using csa::uni::UnionParams;
+    if (rows < 0 || topk <= 0 || T < 0 || cap <= 0 || n_lists < 1 ||
+        n_lists > csa::uni::kMaxLists || !lists)
+        return CSA_ERR_INVALID_ARG;
+    if (rows == 0)
+        return CSA_OK;
+    if (!out || !count || !aligned(out, 4) || !aligned(count, 4))
+        return CSA_ERR_INVALID_ARG;
+    UnionParams p;
+    std::memset(&p, 0, sizeof p);
+    for (int l = 0; l < n_lists; ++l) {
+        if (!lists[l] || !aligned(lists[l], 4))
+            return CSA_ERR_INVALID_ARG;
+        p.lists[l] = lists[l];
+    }
+    p.n_lists = n_lists;
+    p.rows = rows;
+    p.topk = topk;
+    p.T = T;
+    p.cap = cap;
+    p.words = (T + 31) / 32;
+    if (p.words < 1)
+        p.words = 1;
+    const long long smem = (static_cast<long long>(p.words) + csa::uni::kThreads / 32) * 4;
+    if (smem > kSmemLimit)
+        return CSA_ERR_UNSUPPORTED;
+    p.out = out;
+    p.count = count;
+    if (cudaFuncSetAttribute(csa::uni::union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    const int sms = device_sms();
+    if (sms <= 0)
+        return CSA_ERR_CUDA;
+    const int per_sm = smem > kSmemLimit / 2 ? 1 : (smem > kSmemLimit / 4 ? 2 : 4);
+    const int grid = rows < per_sm * sms ? rows : per_sm * sms;
+    csa::uni::union_kernel<<<grid, csa::uni::kThreads, static_cast<int>(smem), stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // Allocation-free entry point.
 //
 // Some callers cannot allocate device memory at call time: serving loops that
@@ -667,6 +840,7 @@ csa_status_t noalloc_scratch(void **out)
 
 extern "C" csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStream_t stream)
 {
+    NvtxRange range("csa_indexer_topk_noalloc");
     csa_status_t st = validate(args);
     if (st != CSA_OK)
         return st;

@@ -36,7 +36,7 @@
 //   warps 12..15 selector
 // The block launches with 128 registers per thread; the two control
 // warpgroups give most of their share to the epilogue warpgroups
-// (4 x 128 x 128 = 2 x 128 x kEpiRegs + 2 x 128 x kCtlRegs).
+// (4 x 128 x 128 = 2 x 128 x kEpiRegs + 128 x kCtlRegs + 128 x kSelRegs).
 //
 // Epilogue fast path (H_I >= 32, at most 128 TMEM columns per warpgroup): a
 // warp reads its 32 TMEM lanes with two 16-lane x 256-bit loads, so every
@@ -61,8 +61,9 @@ constexpr int kSlotCols = 256;   // TMEM columns per accumulator slot
 constexpr int kThreads = 512;
 constexpr int kLaunchRegs = 128;  // registers per thread the kernel must be built with
 constexpr int kEpiRegs = 160;     // after the split: epilogue warpgroups
-constexpr int kCtlRegs = 96;      //                  producer / MMA / splitter, selector
-static_assert(2 * 128 * kEpiRegs + 2 * 128 * kCtlRegs == kThreads * kLaunchRegs,
+constexpr int kCtlRegs = 96;      //                  producer / MMA / splitter
+constexpr int kSelRegs = 96;      //                  selector
+static_assert(2 * 128 * kEpiRegs + 128 * kCtlRegs + 128 * kSelRegs == kThreads * kLaunchRegs,
               "register split must match the launch budget");
 constexpr int kGroupThreads = 128;
 constexpr int kBarWg0 = 1, kBarWg1 = 2, kBarSelect = 3;  // named barriers
@@ -211,20 +212,6 @@ struct Barriers {
     int abort;
 };
 
-// Bounded wait used when unwinding: ignores the abort flag and the (possibly
-// shrunk) per-wait budget, so that copies and MMAs already in flight land
-// before the CTA frees its shared memory and TMEM.  Work in flight finishes in
-// microseconds; the fixed budget (about a second) only bounds a broken GPU.
-constexpr long long kDrainLimit = 1ll << 31;
-
-__device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, long long limit = kDrainLimit)
-{
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > limit)
-            return;
-    }
-}
 
 // Hint: bring [src, src+bytes) into L2 (16-byte aligned, multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
@@ -670,11 +657,13 @@ __device__ __forceinline__ float2 relu2(uint32_t a, uint32_t b)
 
 // Scores of FQ queries for one key per thread.  The warp's two 16-lane loads
 // cover its 32 keys; thread t holds columns 8i + 2(t%4) + {0,1} of keys
-// t/4 + {0, 8, 16, 24}.  After the loads land the accumulator slot is released
-// (one arrive per warp).  Each thread then forms per-key partial sums over its
-// columns (column pairs with one packed FMA); the quad (threads sharing t/4)
-// exchanges halves twice so that thread t ends with the complete scores of
-// key row 16*((t>>1)&1) + 8*(t&1) + t/4 of the warp's 32.
+// t/4 + {0, 8, 16, 24}.  The second load (the warp's upper 16 lanes) is in
+// flight while the first one's columns are reduced, and the accumulator slot
+// is released (one arrive per warp) as soon as it has landed.  Each thread
+// forms per-key partial sums over its columns (column pairs with one packed
+// FMA); the quad (threads sharing t/4) exchanges halves twice so that thread
+// t ends with the complete scores of key row 16*((t>>1)&1) + 8*(t&1) + t/4 of
+// the warp's 32.
 template <int FC, int FQ>
 __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&wr)[FC / 8],
                                                  uint64_t *acc_empty, int lane, float (&F)[FQ])
@@ -683,35 +672,49 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
     constexpr int REPS = FC / 8;
     constexpr int RPQ = REPS / FQ;
     uint32_t va[NV], vb[NV];
-    __syncwarp();
-    Ld16x256<FC>::ld(taddr, va);
-    Ld16x256<FC>::ld(taddr + (16u << 16), vb);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        reg_fence(va[i]);
-        reg_fence(vb[i]);
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0 && acc_empty)
-        mbar_arrive(acc_empty);
     float2 P[4][FQ];
 #pragma unroll
     for (int k = 0; k < 4; ++k)
 #pragma unroll
         for (int j = 0; j < FQ; ++j)
             P[k][j] = make_float2(0.0f, 0.0f);
+    __syncwarp();
+    Ld16x256<FC>::ld(taddr, va);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+        reg_fence(va[i]);
+    Ld16x256<FC>::ld(taddr + (16u << 16), vb);      // lands while va is reduced
 #pragma unroll
     for (int i = 0; i < REPS; ++i) {
         const int j = i / RPQ;
 #pragma unroll
-        for (int sub = 0; sub < 2; ++sub) {
+        for (int sub = 0; sub < 2; ++sub)
             P[sub][j] = __ffma2_rn(relu2(va[4 * i + 2 * sub], va[4 * i + 2 * sub + 1]), wr[i],
                                    P[sub][j]);
+    }
+#pragma unroll
+    for (int j = 0; j < FQ; ++j) {                  // va's sums are formed before the wait
+        fence_f32(P[0][j].x);
+        fence_f32(P[0][j].y);
+        fence_f32(P[1][j].x);
+        fence_f32(P[1][j].y);
+    }
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+        reg_fence(vb[i]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0 && acc_empty)
+        mbar_arrive(acc_empty);
+#pragma unroll
+    for (int i = 0; i < REPS; ++i) {
+        const int j = i / RPQ;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub)
             P[2 + sub][j] = __ffma2_rn(relu2(vb[4 * i + 2 * sub], vb[4 * i + 2 * sub + 1]), wr[i],
                                        P[2 + sub][j]);
-        }
     }
     const bool b1 = (lane >> 1) & 1;
     const bool b0 = lane & 1;
@@ -1357,7 +1360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (warp >= 10 && p.key_fp8)
             run_qsplit(p, smem, bars, ctl, threadIdx.x - 320);
     } else {
-        regs_dec<kCtlRegs>();
+        regs_dec<kSelRegs>();
         run_selector(p, smem, bars, ctl);
     }
 

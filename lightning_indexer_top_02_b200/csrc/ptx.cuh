@@ -111,6 +111,21 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, con
     }
 }
 
+// Bounded wait used when unwinding: ignores the abort flag and the (possibly
+// shrunk) per-wait budget, so that copies and MMAs already in flight land
+// before the CTA frees its shared memory and TMEM.  Work in flight finishes in
+// microseconds; the fixed budget (about a second) only bounds a broken GPU.
+constexpr long long kDrainLimit = 1ll << 31;
+
+__device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, long long limit = kDrainLimit)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit)
+            return;
+    }
+}
+
 // ---------------------------------------------------------------- register split
 // Moves registers between warpgroups: every warp of a warpgroup executes the
 // same call.  An increase waits until enough registers have been released by
@@ -141,6 +156,20 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Four rows of a 2-D tensor (row coordinates r0..r3, any order, the box one
+// row high) from column c0 into consecutive rows at dst, swizzled as the
+// tensor map says.
+__device__ __forceinline__ void tma_gather4(void *dst, const void *tmap, uint64_t *bar, int c0,
+                                            int r0, int r1, int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -283,11 +312,38 @@ __device__ __forceinline__ void tmem_ld_wait()
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 lanes x 32 consecutive 32-bit columns: thread (lane) writes its row's 32 values.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Ties a register to program order after tmem_ld_wait(), so no use of it can be
 // scheduled before the load has landed.
 __device__ __forceinline__ void reg_fence(uint32_t &r)
 {
     asm volatile("" : "+r"(r));
+}
+
+// Ties a value to program order: it is computed before any later volatile asm
+// (e.g. a wait that should overlap with the arithmetic that produces it).
+__device__ __forceinline__ void fence_f32(float &x)
+{
+    asm volatile("" : "+f"(x));
 }
 
 // ---------------------------------------------------------------- descriptors
@@ -303,6 +359,18 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, int row_byt
     const uint64_t sbo = static_cast<uint64_t>(8 * row_bytes) >> 4;
     return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (sbo << 32) |
            (1ull << 46) | (layout << 61);
+}
+
+// Shared-memory matrix descriptor for an MN-major operand with 128-byte
+// swizzle: each 128-byte row holds 64 consecutive MN elements at one K index,
+// 8 K rows form a 1024-byte atom (sbo_bytes between atoms along K), and the
+// next 64 MN elements start lbo_bytes further on.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                       uint32_t sbo_bytes)
+{
+    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) |
+           (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
 // Instruction descriptor: D fp32, A and B both bf16 (ab_bf16=1) or both f16,

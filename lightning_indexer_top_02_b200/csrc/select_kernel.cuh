@@ -210,21 +210,12 @@ __device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_li
     return prefix;
 }
 
-// Bucket of a score image: integer ranges of the image when every key has the
-// same sign (the image is then roughly logarithmic in the score, which spreads
-// the dense scores just above a cut), linear in the score otherwise.
-struct SelMap {
-    uint32_t mn;
-    int shift;
-    bool by_ord;
-    BucketMap bm;
-};
-
-__device__ __forceinline__ int sel_bucket(uint32_t o, const SelMap &m)
+// Bucket of a score image over the row's own [min, max], numbered from the
+// top score down (range_map: integer ranges of the image when every key has
+// the same sign, linear in the score otherwise).
+__device__ __forceinline__ int sel_bucket(uint32_t o, const RangeMap &m)
 {
-    if (m.by_ord)
-        return kSelNb - 1 - static_cast<int>((o - m.mn) >> m.shift);
-    return kSelNb - 1 - bucket_of(score_of_ord(o), m.bm, kSelNb);
+    return kSelNb - 1 - range_bucket(o, m, kSelNb);
 }
 
 __device__ __forceinline__ void sel_store(int32_t *oi, float *os, int slot, uint64_t key)
@@ -262,14 +253,9 @@ __device__ void sel_sort_regs(SelSmem *sm, const uint64_t (&e)[kSelEpt], int n, 
         mn = min(mn, sm->gs.warp_sums[w]);
         mx = max(mx, sm->gs.warp_sums[16 + w]);
     }
-    SelMap map;
-    map.mn = mn;
-    map.by_ord = (mn >> 31) == (mx >> 31);
-    const uint32_t span = mx - mn;
-    map.shift = span < static_cast<uint32_t>(kSelNb) ? 0 : 32 - __clz(span) - 11;
-    map.bm = bucket_map(mn, mx, kSelNb);
+    const RangeMap map = range_map(mn, mx, kSelNb);
     int total = n;
-    bool fallback = mx == mn || (!map.by_ord && !map.bm.ok);
+    bool fallback = !map.ok;
     if (!fallback) {
         // histogram, buckets numbered from the top score down
         int db[kSelEpt];

@@ -142,6 +142,74 @@ __device__ __forceinline__ int bucket_of(float s, const BucketMap &m, int NB)
     return b > NB - 1 ? NB - 1 : b;
 }
 
+// Monotone map of score images in [lo, hi] onto NB buckets (NB a power of
+// two), ascending with the score: integer ranges of the image when both ends
+// share a sign (the image is then roughly logarithmic in the score, which
+// spreads the dense scores just above a cut), linear in the score otherwise.
+// ok is false when every score is equal or the range is not finite.
+struct RangeMap {
+    uint32_t mn;
+    int shift;
+    bool by_ord;
+    bool ok;
+    BucketMap bm;
+};
+
+__device__ __forceinline__ RangeMap range_map(uint32_t lo, uint32_t hi, int NB)
+{
+    RangeMap m;
+    m.mn = lo;
+    m.by_ord = (lo >> 31) == (hi >> 31);
+    const uint32_t span = hi - lo;
+    const int nb_bits = 31 - __clz(NB);
+    m.shift = span < static_cast<uint32_t>(NB) ? 0 : 32 - __clz(span) - nb_bits;
+    m.bm = bucket_map(lo, hi, NB);
+    m.ok = hi > lo && (m.by_ord || m.bm.ok);
+    return m;
+}
+
+__device__ __forceinline__ int range_bucket(uint32_t o, const RangeMap &m, int NB)
+{
+    if (m.by_ord) {
+        const uint32_t b = (o > m.mn ? o - m.mn : 0u) >> m.shift;
+        return b > static_cast<uint32_t>(NB - 1) ? NB - 1 : static_cast<int>(b);
+    }
+    return bucket_of(score_of_ord(o), m.bm, NB);
+}
+
+// The smallest score image in [lo, hi] whose bucket is at least b (b at most
+// the bucket of hi): every image at or above it maps to b or higher, every
+// image below it to a lower bucket.  Integer ranges: the bucket's first
+// image.  Linear ranges: the image of the bucket's lower edge, moved to the
+// exact boundary by a few one-ulp steps (bisection if rounding put it far).
+__device__ __forceinline__ uint32_t range_bucket_floor(uint32_t lo, uint32_t hi, int b,
+                                                       const RangeMap &m, int NB)
+{
+    if (m.by_ord) {
+        const unsigned long long f = static_cast<unsigned long long>(m.mn) +
+                                     (static_cast<unsigned long long>(b) << m.shift);
+        return f < lo ? lo : (f > hi ? hi : static_cast<uint32_t>(f));
+    }
+    uint32_t o = ord_of_score(m.bm.lo + static_cast<float>(b) / m.bm.inv);
+    o = o < lo ? lo : (o > hi ? hi : o);
+    for (int step = 0; step < 16; ++step) {
+        if (o > lo && range_bucket(o - 1, m, NB) >= b)
+            --o;
+        else if (o < hi && range_bucket(o, m, NB) < b)
+            ++o;
+        else
+            return o;
+    }
+    while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (range_bucket(mid, m, NB) >= b)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    return lo;
+}
+
 __host__ __device__ constexpr int pow2_at_least(int x)
 {
     int p = 2;
