@@ -256,6 +256,41 @@ def config_dict(wl):
             "parallelism": "replicas"}
 
 
+# ----------------------------------------------------------------------------- consumer leg
+def attention_leg(L, wl, out_idx, dev, stream, steps, warmup, HA=64, Dk=128, Dv=128):
+    """Sparse attention over the selection the timed indexer steps produced:
+    CUDA-event time per call, algorithmic flops (2 HA (Dk + Dv) per selected
+    key) and gathered bytes (each selected key's cache row read once per query,
+    plus q and the output)."""
+    import torch
+
+    g = torch.Generator(device=dev).manual_seed(7)
+    qa = torch.randn((wl.B, wl.S, HA, Dk), generator=g, device=dev).to(torch.bfloat16)
+    kc = torch.randn((wl.B, wl.T, Dk), generator=g, device=dev).to(torch.bfloat16)
+    vc = torch.randn((wl.B, wl.T, Dv), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((wl.B, wl.S, HA, Dv), dtype=torch.float32, device=dev)
+    n_sel = int((out_idx >= 0).sum().item())
+    for _ in range(warmup):
+        L.sparse_attention(qa, kc, out_idx, scale=Dk ** -0.5, v=vc, out=out, stream=stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e0, e1 in ev:
+        e0.record(stream)
+        L.sparse_attention(qa, kc, out_idx, scale=Dk ** -0.5, v=vc, out=out, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if L.csa_last_device_error(None) != L.CSA_OK:
+        raise SystemExit("device error in the attention leg")
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    flops = 2.0 * HA * (Dk + Dv) * n_sel
+    gathered = n_sel * (Dk + Dv) * 2 + qa.numel() * 2 + out.numel() * 4
+    return {"kernel": "sparse_attn_kernel", "heads": HA, "Dk": Dk, "Dv": Dv,
+            "selected_keys": n_sel, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+            "gathered_gbs": gathered / (ms * 1e-3) / 1e9,
+            "queries_per_s": wl.B * wl.S / (ms * 1e-3)}
+
+
 # ----------------------------------------------------------------------------- GPU leg
 def main():
     ap = argparse.ArgumentParser()
@@ -274,6 +309,9 @@ def main():
     ap.add_argument("--clocks-csv", default="",
                     help="keep the raw nvidia-smi clock samples of the timed region here")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attention", action="store_true",
+                    help="also time the sparse-attention consumer over the step's selection "
+                         "(HA=64 heads, Dk=Dv=128, bf16; reported under 'consumer')")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -498,6 +536,9 @@ def main():
                           "ms_per_step": serial_ms,
                           "what": "upload, call and read-back of each step in series on one stream"}}
 
+    consumer = attention_leg(L, wl, out_idx, dev, stream, args.steps, args.warmup) \
+        if args.attention else None
+
     if rank != 0:
         if world > 1:
             dist.barrier()
@@ -563,6 +604,7 @@ def main():
         "data": "synthetic", "config": config_dict(wl), "tflops": tflops,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * plan.launches,
+        **({"consumer": consumer} if consumer else {}),
         "plan": plan.as_dict(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
                     "max": max(step_ms)},

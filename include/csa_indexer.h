@@ -72,6 +72,9 @@ typedef enum {
 } csa_status_t;
 
 typedef enum { CSA_KEY_BF16 = 0, CSA_KEY_E4M3 = 1 } csa_key_dtype_t;
+
+/* q_offset value that selects the default alignment max(0, T*m - S). */
+#define CSA_Q_OFFSET_DEFAULT (-9223372036854775807LL - 1)
 typedef enum { CSA_MODE_TOPK = 0, CSA_MODE_GATE = 1 } csa_mode_t;
 
 /* Full argument set of one indexer call.  Pointers are device pointers. */
@@ -84,9 +87,10 @@ typedef struct {
     int causal;            /* 0: every key visible; 1: the causal rule above   */
     int key_dtype;         /* csa_key_dtype_t                                  */
     int mode;              /* csa_mode_t                                       */
-    long long q_offset;    /* absolute position of query row 0; < 0 selects the
-                              default max(0, T*m - S) (queries end where the
-                              keys' token span ends)                           */
+    long long q_offset;    /* absolute position of query row 0 (may be
+                              negative: rows before position 0 see no key);
+                              CSA_Q_OFFSET_DEFAULT selects max(0, T*m - S)
+                              (queries end where the keys' token span ends)  */
     int num_splits;        /* key-range splits per query block; 0 = automatic  */
     int32_t *out_idx;      /* [B,S,topk]                                       */
     float *out_score;      /* [B,S,topk]                                       */
@@ -194,6 +198,28 @@ typedef struct {
 } csa_attn_args_t;
 
 csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaStream_t stream);
+
+/*
+ * Exact merge of top-k lists made over disjoint key ranges, e.g. one list per
+ * GPU when the keys are sharded across GPUs ("Million-Token Memory Without
+ * the Global Bottleneck": keys split across GPUs, a selection on each, then
+ * a combination that covers the global top).  idx and score are HOST arrays
+ * of n_lists (1..64) DEVICE pointers, each [rows, k_in] (an indexer's
+ * out_idx / out_score over its key range); key_offset is a HOST array of
+ * n_lists offsets added to each list's indices (the first key of its range),
+ * and entries with index < 0 are padding.  out_idx / out_score [rows, topk]
+ * receive the topk largest scores of the union, ordered by score descending,
+ * equal scores by ascending (offset) index, padded with -1 / -inf.  When
+ * every list holds its range's top min(topk, k_in) keys with k_in >= topk,
+ * this is exactly the top-k over all ranges.  workspace: device memory of
+ * csa_merge_workspace_size(n_lists, rows, k_in) bytes, 256-byte aligned, or
+ * NULL to allocate stream-ordered.  topk <= 2048.
+ */
+csa_status_t csa_merge_topk(const int32_t *const *idx, const float *const *score,
+                            const long long *key_offset, int n_lists, int rows, int k_in,
+                            int topk, int32_t *out_idx, float *out_score, void *workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+size_t csa_merge_workspace_size(int n_lists, int rows, int k_in);
 
 /*
  * OR-union of several layers' selections ("FlashMemory-DeepSeek-V4:

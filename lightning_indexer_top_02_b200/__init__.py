@@ -35,10 +35,11 @@ CSA_KEY_BF16 = 0
 CSA_KEY_E4M3 = 1
 CSA_MODE_TOPK = 0
 CSA_MODE_GATE = 1
+CSA_Q_OFFSET_DEFAULT = -(1 << 63)
 
 EXPORTS = ("csa_indexer_topk", "csa_indexer_topk_ex", "csa_indexer_workspace_size",
            "csa_indexer_plan", "csa_indexer_topk_noalloc", "csa_sparse_attention",
-           "csa_union_selections",
+           "csa_union_selections", "csa_merge_topk", "csa_merge_workspace_size",
            "csa_status_string", "csa_last_device_error", "csa_set_wait_limit",
            "csa_set_launch_events", "csa_version")
 
@@ -103,6 +104,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.csa_indexer_workspace_size.restype = ctypes.c_size_t
     lib.csa_indexer_topk_noalloc.argtypes = [ctypes.POINTER(CsaArgs), P]
     lib.csa_indexer_topk_noalloc.restype = I
+    lib.csa_merge_topk.argtypes = [P, P, P, I, I, I, I, P, P, P, ctypes.c_size_t, P]
+    lib.csa_merge_topk.restype = I
+    lib.csa_merge_workspace_size.argtypes = [I, I, I]
+    lib.csa_merge_workspace_size.restype = ctypes.c_size_t
     lib.csa_union_selections.argtypes = [P, I, I, I, I, I, P, P, P]
     lib.csa_union_selections.restype = I
     lib.csa_sparse_attention.argtypes = [ctypes.POINTER(CsaAttnArgs), P]
@@ -196,7 +201,7 @@ def _ptr(t):
 
 
 def make_args(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
-              mode: int = CSA_MODE_TOPK, q_offset: int = -1, num_splits: int = 0,
+              mode: int = CSA_MODE_TOPK, q_offset: Optional[int] = None, num_splits: int = 0,
               query_pieces: int = 0, out_idx=None, out_score=None) -> CsaArgs:
     """Pack torch tensors into the C argument struct (shapes read from q and k)."""
     import torch
@@ -211,7 +216,7 @@ def make_args(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
     a.causal = int(bool(causal))
     a.key_dtype = CSA_KEY_E4M3 if fp8 else CSA_KEY_BF16
     a.mode = int(mode)
-    a.q_offset = int(q_offset)
+    a.q_offset = CSA_Q_OFFSET_DEFAULT if q_offset is None else int(q_offset)
     a.num_splits = int(num_splits)
     a.query_pieces = int(query_pieces)
     a.out_idx = out_idx.data_ptr() if out_idx is not None else None
@@ -220,8 +225,9 @@ def make_args(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
 
 
 def indexer_topk(q, w, k, *, k_scale=None, m: int, topk: int, causal: bool = True,
-                 mode: int = CSA_MODE_TOPK, q_offset: int = -1, num_splits: int = 0,
-                 query_pieces: int = 0, out_idx=None, out_score=None, workspace=None,
+                 mode: int = CSA_MODE_TOPK, q_offset: Optional[int] = None,
+                 num_splits: int = 0, query_pieces: int = 0, out_idx=None, out_score=None,
+                 workspace=None,
                  stream=None):
     """Run the indexer top-k on CUDA tensors; returns (out_idx, out_score).
 

@@ -123,6 +123,9 @@ csa_status_t validate(const csa_args_t *a)
         !aligned(a->out_idx, 4) || !aligned(a->out_score, 4) ||
         (a->k_scale && !aligned(a->k_scale, 4)))
         return CSA_ERR_INVALID_ARG;
+    if (a->q_offset != CSA_Q_OFFSET_DEFAULT &&
+        (a->q_offset < -(1ll << 62) || a->q_offset > (1ll << 62)))
+        return CSA_ERR_INVALID_ARG;
     if (!is_pow2(a->H_I) || a->H_I > 256)
         return CSA_ERR_UNSUPPORTED;
     if (a->d != 32 && a->d != 64 && a->d != 128)
@@ -176,7 +179,7 @@ csa_status_t make_plan(const csa_args_t *a, int sms, size_t ws_cap, Plan *out)
     p.mode = a->mode;
     p.key_fp8 = a->key_dtype == CSA_KEY_E4M3;
     p.q_pieces = p.key_fp8 ? (a->query_pieces == 1 ? 1 : 2) : 0;
-    p.q_offset = a->q_offset >= 0 ? a->q_offset
+    p.q_offset = a->q_offset != CSA_Q_OFFSET_DEFAULT ? a->q_offset
                                   : (static_cast<long long>(a->T) * a->m > a->S
                                          ? static_cast<long long>(a->T) * a->m - a->S
                                          : 0);
@@ -586,7 +589,7 @@ csa_status_t csa_indexer_topk(const void *q, const float *w, const void *k, int 
     a.causal = causal;
     a.key_dtype = CSA_KEY_BF16;
     a.mode = CSA_MODE_TOPK;
-    a.q_offset = -1;
+    a.q_offset = CSA_Q_OFFSET_DEFAULT;
     a.num_splits = 0;
     a.query_pieces = 0;
     a.out_idx = out_idx;
@@ -750,6 +753,158 @@ extern "C" csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaSt
     if (!mark(1, stream))
         return CSA_ERR_CUDA;
     return CSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Exact merge of top-k lists over disjoint key ranges (key shards).
+namespace {
+
+// One CTA per (row, list): the list's valid entries (index >= 0), in order,
+// as 64-bit keys (score image << 32 | ~(index + offset)) in the select
+// kernel's list layout, and their count.
+__global__ void __launch_bounds__(256) pack_lists_kernel(csa::SelParams sp, const int32_t *const *idx,
+                                                         const float *const *score,
+                                                         const long long *offset, int k_in,
+                                                         uint64_t *lists, int *counts)
+{
+    __shared__ int warp_tot[8];
+    const int r = blockIdx.x / sp.nsplit, l = blockIdx.x % sp.nsplit;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int32_t *src_i = idx[l] + static_cast<size_t>(r) * k_in;
+    const float *src_s = score[l] + static_cast<size_t>(r) * k_in;
+    uint64_t *dst = lists + (static_cast<size_t>(r) * sp.nsplit + l) * sp.cap;
+    int base = 0;
+    for (int j0 = 0; j0 < k_in; j0 += 256) {
+        const int j = j0 + tid;
+        const int32_t s = j < k_in ? src_i[j] : -1;
+        const bool ok = s >= 0;
+        const uint32_t m = __ballot_sync(0xffffffffu, ok);
+        if (lane == 0)
+            warp_tot[wid] = __popc(m);
+        __syncthreads();
+        int before = 0, tot = 0;
+        for (int w = 0; w < 8; ++w) {
+            before += w < wid ? warp_tot[w] : 0;
+            tot += warp_tot[w];
+        }
+        if (ok) {
+            const long long g = static_cast<long long>(s) + offset[l];
+            dst[base + before + __popc(m & ((1u << lane) - 1u))] =
+                csa::make_key(csa::ord_of_score(src_s[j]), static_cast<uint32_t>(g));
+        }
+        base += tot;
+        __syncthreads();
+    }
+    if (tid == 0)
+        counts[static_cast<size_t>(r) * sp.nsplit + l] = base;
+}
+
+size_t merge_lists_bytes(int n_lists, int rows, int k_in)
+{
+    return align256(static_cast<size_t>(rows) * n_lists * k_in * 8);
+}
+
+size_t merge_ws_bytes(int n_lists, int rows, int k_in)
+{
+    return merge_lists_bytes(n_lists, rows, k_in) + align256(static_cast<size_t>(rows) * n_lists * 4) +
+           align256(static_cast<size_t>(n_lists) * (2 * sizeof(void *) + sizeof(long long)));
+}
+
+} // namespace
+
+extern "C" size_t csa_merge_workspace_size(int n_lists, int rows, int k_in)
+{
+    if (n_lists < 1 || n_lists > csa::kSelMaxSplits || rows < 0 || k_in < 1)
+        return 0;
+    return merge_ws_bytes(n_lists, rows, k_in);
+}
+
+extern "C" csa_status_t csa_merge_topk(const int32_t *const *idx, const float *const *score,
+                                       const long long *key_offset, int n_lists, int rows,
+                                       int k_in, int topk, int32_t *out_idx, float *out_score,
+                                       void *workspace, size_t workspace_bytes,
+                                       cudaStream_t stream)
+{
+    NvtxRange range("csa_merge_topk");
+    if (!idx || !score || !key_offset || n_lists < 1 || n_lists > csa::kSelMaxSplits ||
+        rows < 0 || k_in < 1 || topk < 1)
+        return CSA_ERR_INVALID_ARG;
+    if (topk > csa::kMaxTopk)
+        return CSA_ERR_UNSUPPORTED;
+    if (rows == 0)
+        return CSA_OK;
+    if (!out_idx || !out_score || !aligned(out_idx, 4) || !aligned(out_score, 4))
+        return CSA_ERR_INVALID_ARG;
+    for (int l = 0; l < n_lists; ++l) {
+        if (!idx[l] || !score[l] || !aligned(idx[l], 4) || !aligned(score[l], 4) ||
+            key_offset[l] < 0 || key_offset[l] + k_in >= (1ll << 31))
+            return CSA_ERR_INVALID_ARG;
+    }
+    const size_t need = merge_ws_bytes(n_lists, rows, k_in);
+    void *ws = workspace;
+    if (ws) {
+        if (workspace_bytes < need)
+            return CSA_ERR_WORKSPACE;
+        if (!aligned(ws, 256))
+            return CSA_ERR_INVALID_ARG;
+    } else if (cudaMallocAsync(&ws, need, stream) != cudaSuccess) {
+        return CSA_ERR_CUDA;
+    }
+    // the list pointers and offsets go to the device through the workspace tail
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    uint64_t *lists = reinterpret_cast<uint64_t *>(w8);
+    int *counts = reinterpret_cast<int *>(w8 + merge_lists_bytes(n_lists, rows, k_in));
+    uint8_t *tail = w8 + merge_lists_bytes(n_lists, rows, k_in) +
+                    align256(static_cast<size_t>(rows) * n_lists * 4);
+    const int32_t **d_idx = reinterpret_cast<const int32_t **>(tail);
+    const float **d_score = reinterpret_cast<const float **>(tail + n_lists * sizeof(void *));
+    long long *d_off = reinterpret_cast<long long *>(tail + 2 * n_lists * sizeof(void *));
+    csa_status_t st = CSA_OK;
+    if (cudaMemcpyAsync(d_idx, idx, n_lists * sizeof(void *), cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(d_score, score, n_lists * sizeof(void *), cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(d_off, key_offset, n_lists * sizeof(long long), cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+        st = CSA_ERR_CUDA;
+    csa::SelParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.lists = lists;
+    sp.counts = counts;
+    sp.rows = rows;
+    sp.nsplit = n_lists;
+    sp.cap = k_in;
+    sp.topk = topk;
+    sp.B = 1;
+    sp.S = rows;
+    sp.qps = 1;
+    sp.nqb = rows;
+    sp.qb_lo = 0;
+    sp.out_idx = out_idx;
+    sp.out_score = out_score;
+    if (st == CSA_OK) {
+        pack_lists_kernel<<<static_cast<unsigned>(rows) * n_lists, 256, 0, stream>>>(
+            sp, d_idx, d_score, d_off, k_in, lists, counts);
+        if (cudaGetLastError() != cudaSuccess)
+            st = CSA_ERR_CUDA;
+    }
+    const int sel_smem = static_cast<int>(sizeof(csa::SelSmem)) + 16;
+    if (st == CSA_OK && cudaFuncSetAttribute(csa::select_topk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             sel_smem) != cudaSuccess)
+        st = CSA_ERR_CUDA;
+    const int sms = device_sms();
+    if (st == CSA_OK && sms <= 0)
+        st = CSA_ERR_CUDA;
+    if (st == CSA_OK) {
+        const int slots = csa::kSelCtasPerSm * sms;
+        csa::select_topk_kernel<<<rows < slots ? rows : slots, csa::kSelThreads, sel_smem, stream>>>(sp);
+        if (cudaGetLastError() != cudaSuccess)
+            st = CSA_ERR_CUDA;
+    }
+    if (!workspace && cudaFreeAsync(ws, stream) != cudaSuccess && st == CSA_OK)
+        st = CSA_ERR_CUDA;
+    return st;
 }
 
 // ---------------------------------------------------------------------------

@@ -23,7 +23,7 @@ def lib():
     return L
 
 
-def run_gpu(L, inp, wl, *, mode=0, q_offset=-1, num_splits=0):
+def run_gpu(L, inp, wl, *, mode=0, q_offset=None, num_splits=0):
     q = inp["q"].cuda()
     w = inp["w"].cuda()
     k = inp["k"].cuda()
@@ -41,10 +41,10 @@ def run_oracle(inp, wl, *, mode=0, q_offset=None, rows=None):
                        topk=wl.topk, causal=wl.causal, mode=mode, q_offset=q_offset, rows=rows)
 
 
-def exact_case(L, wl, *, mode=0, q_offset=-1, num_splits=0, seed=None):
+def exact_case(L, wl, *, mode=0, q_offset=None, num_splits=0, seed=None):
     inp = workloads.make_inputs(wl.replace(values="integer"), seed=seed)
     gi, gs = run_gpu(L, inp, wl, mode=mode, q_offset=q_offset, num_splits=num_splits)
-    ri, rs, _, _ = run_oracle(inp, wl, mode=mode, q_offset=None if q_offset < 0 else q_offset)
+    ri, rs, _, _ = run_oracle(inp, wl, mode=mode, q_offset=q_offset)
     check_exact(gi.reshape(-1, wl.topk), gs.reshape(-1, wl.topk), ri, rs, label=str(wl))
 
 
@@ -88,7 +88,7 @@ def test_splits_bit_exact(lib, num_splits):
     exact_case(lib, wl, num_splits=num_splits)
 
 
-@pytest.mark.parametrize("q_offset", [0, 37, 11000])
+@pytest.mark.parametrize("q_offset", [0, 37, 11000, -60])
 def test_q_offset_bit_exact(lib, q_offset):
     wl = workloads.Workload("o", B=1, S=129, T=2800, H=32, d=64, m=4, topk=64, values="integer", seed=700)
     exact_case(lib, wl, q_offset=q_offset)

@@ -88,7 +88,7 @@ def test_too_large_is_refused(lib):
     the call must refuse before launching anything."""
     a = lib.CsaArgs()
     a.B, a.S, a.T, a.H_I, a.d, a.m, a.topk = 1024, 4, 8192, 64, 128, 4, 2048
-    a.causal, a.q_offset = 1, -1
+    a.causal, a.q_offset = 1, lib.CSA_Q_OFFSET_DEFAULT
     a.q = a.w = a.k = a.out_idx = a.out_score = 1 << 20  # never dereferenced
     st = lib.csa_indexer_topk_noalloc(a, None)
     assert st == lib.CSA_ERR_WORKSPACE
