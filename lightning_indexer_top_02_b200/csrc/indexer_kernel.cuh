@@ -735,6 +735,58 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
     }
 }
 
+// The fast tile math in chunks, for the software pipeline across tiles.  A
+// chunk is one 16-lane x 64-column TMEM load (16x256b.x8, 32 registers):
+// half h (0: the warp's lanes 0-15, 1: lanes 16-31) and column group cg (64
+// columns = repetitions 8cg .. 8cg+7 of the tile's FC/8).  ft_chunk adds a
+// chunk's ReLU(logit) x weight pairs to the per-key partial sums; ft_finish
+// leaves each thread its key's FQ scores.
+template <int FC, int FQ>
+__device__ __forceinline__ void ft_chunk(const uint32_t (&x)[32], const float2 (&wr)[FC / 8],
+                                         float2 (&P)[4][FQ], int h, int cg)
+{
+    constexpr int RPQ = (FC / 8) / FQ;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int i = 8 * cg + r;
+        const int j = i / RPQ;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub)
+            P[2 * h + sub][j] =
+                __ffma2_rn(relu2(x[4 * r + 2 * sub], x[4 * r + 2 * sub + 1]), wr[i], P[2 * h + sub][j]);
+    }
+}
+
+template <int FQ>
+__device__ __forceinline__ void ft_finish(const float2 (&P)[4][FQ], int lane, float (&F)[FQ])
+{
+    const bool b1 = (lane >> 1) & 1;
+    const bool b0 = lane & 1;
+#pragma unroll
+    for (int j = 0; j < FQ; ++j) {
+        float R[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const float lo = P[m][j].x + P[m][j].y;          // key m (first 16 lanes)
+            const float hi = P[2 + m][j].x + P[2 + m][j].y;  // key 2+m (last 16 lanes)
+            const float send = b1 ? lo : hi;
+            const float keep = b1 ? hi : lo;
+            R[m] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        }
+        const float send = b0 ? R[0] : R[1];
+        const float keep = b0 ? R[1] : R[0];
+        F[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+}
+
+// TMEM address of chunk c (of NC = 2 * FC/64) of a tile: halves outermost.
+template <int FC>
+__device__ __forceinline__ uint32_t ft_chunk_addr(uint32_t tile_addr, int c)
+{
+    constexpr int CGS = FC / 64;
+    return tile_addr + ((c / CGS) ? (16u << 16) : 0u) + 64u * static_cast<uint32_t>(c % CGS);
+}
+
 // ------------------------------------------------------------------ generic tile math
 // One 32-column TMEM chunk: sum over the chunk's heads of w * ReLU(logit),
 // four independent accumulators.
@@ -858,6 +910,117 @@ __device__ void run_epilogue(const Params &p, uint8_t *smem, Barriers *bars, uin
             break;
         float *buf = p.scores + (static_cast<size_t>(blockIdx.x) * 2 + par) * p.qps * p.nmax +
                      static_cast<size_t>(j0) * p.nmax;
+
+        if constexpr (FC > 0) {
+            if (p.tpg == 1 && !p.tile_split) {
+                // One tile per accumulator slot: a software pipeline across the
+                // item's tiles in chunks of 16 lanes x 64 columns, two buffers of
+                // 32 registers: the next chunk (of this tile, or the first of the
+                // next tile) loads while the current one is reduced.  The slot
+                // goes back to the MMA once the tile's last chunk has landed.
+                constexpr int NC = 2 * (FC / 64);
+                uint32_t xa[32], xb[32];
+                const uint32_t lane_base =
+                    tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
+                int slot = 0;
+                if (it.tile_begin < it.tile_end) {
+                    slot = acc_use & 1;
+                    pf.start();
+                    ok = wait_bounded(&bars->acc_full[slot], (acc_use >> 1) & 1, ctl,
+                                      kRoleEpilogue, id);
+                    ok = __all_sync(0xffffffffu, ok);
+                    pf.add(pa, kPfEpiAccFull, rec);
+                    ++acc_use;
+                    if (ok) {
+                        tc_fence_after();
+                        __syncwarp();
+                        tmem_ld_16x256b_x8(ft_chunk_addr<FC>(lane_base + slot * kSlotCols, 0), xa);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            reg_fence(xa[i]);
+                    }
+                }
+                for (int t = it.tile_begin; t < it.tile_end && ok; ++t) {
+                    pf.count(pa, kPfEpiTiles, rec);
+                    const int s = t * kTileKeys + key_local;
+                    const size_t off = static_cast<size_t>(t - it.tile_begin) * kTileKeys + key_local;
+                    float kscale = 1.0f;
+                    if (p.key_fp8 && s < p.T)
+                        kscale = p.k_scale[static_cast<size_t>(it.b) * p.T + s];
+                    const bool in_buf = CSA_CHECK_INDEX(kChkScoreBuf, off, p.nmax);
+                    (void)in_buf;
+                    pf.start();
+                    const uint32_t tile_addr = lane_base + slot * kSlotCols;
+                    const bool next = t + 1 < it.tile_end;
+                    float2 P[4][FQ];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+#pragma unroll
+                        for (int j = 0; j < FQ; ++j)
+                            P[k][j] = make_float2(0.0f, 0.0f);
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) {
+                        uint32_t(&cur)[32] = (c & 1) ? xb : xa;
+                        uint32_t(&nxt)[32] = (c & 1) ? xa : xb;
+                        bool more = true;
+                        if (c + 1 < NC) {
+                            tmem_ld_16x256b_x8(ft_chunk_addr<FC>(tile_addr, c + 1), nxt);
+                        } else {
+                            // every chunk of tile t has landed: the slot is free
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive(&bars->acc_empty[slot]);
+                            more = next;
+                            if (next) {
+                                slot = acc_use & 1;
+                                ok = wait_bounded(&bars->acc_full[slot], (acc_use >> 1) & 1, ctl,
+                                                  kRoleEpilogue, id);
+                                ok = __all_sync(0xffffffffu, ok);
+                                ++acc_use;
+                                more = ok;
+                                if (ok) {
+                                    tc_fence_after();
+                                    __syncwarp();
+                                    tmem_ld_16x256b_x8(
+                                        ft_chunk_addr<FC>(lane_base + slot * kSlotCols, 0), nxt);
+                                }
+                            }
+                        }
+                        ft_chunk<FC, FQ>(cur, wr, P, c / (FC / 64), c % (FC / 64));
+#pragma unroll
+                        for (int j = 0; j < FQ; ++j) {   // the sums are formed before the wait
+                            fence_f32(P[0][j].x);
+                            fence_f32(P[1][j].x);
+                            fence_f32(P[2][j].x);
+                            fence_f32(P[3][j].x);
+                        }
+                        if (more) {
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                reg_fence(nxt[i]);
+                        }
+                    }
+                    float F[FQ];
+                    ft_finish<FQ>(P, lane, F);
+#pragma unroll
+                    for (int q = 0; q < FQ; ++q)
+                        if (in_buf)
+                            buf[static_cast<size_t>(q) * p.nmax + off] = F[q] * kscale;
+                    pf.add(pa, kPfEpiMath, rec);
+                }
+                // Hand this half to the selector (one arrive per warp).
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->buf_full[par]);
+                if (!ok)
+                    *ctl.abort = 1;
+                ++it_count;
+                continue;
+            }
+        }
 
         int slot = 0;      // accumulator slot of the current tile group
         bool mine = true;  // tile_split: the current group is this warpgroup's
