@@ -165,9 +165,10 @@ csa_status_t csa_indexer_topk_noalloc(const csa_args_t *args, cudaStream_t strea
  * via Streaming Top-k", abstract: a sparse attention kernel reads only the
  * selected compressed keys).  For every batch b, query row i and head g < HA:
  *
- *   J = idx[b,i,0..n), the selected keys, where n is the first slot that holds
- *       no key in [0, T) (the indexer lists its selection first and pads with
- *       -1; anything after the first such slot is ignored)
+ *   J = the entries of idx[b,i,0..topk) that lie in [0, T), in slot order
+ *       (the indexer lists its selection first and pads with -1; an entry
+ *       outside [0, T) is padding wherever it stands, and the slots after the
+ *       last key are not read twice)
  *   out[b,i,g,:] = sum_j softmax_j( scale * q[b,i,g,:] . k[b,J_j,:] ) * v[b,J_j,:]
  *   (zeros when n = 0)
  *

@@ -710,19 +710,27 @@ extern "C" csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaSt
     p.idx = args->idx;
     p.out = args->out;
     p.wait_limit = static_cast<long long>(g_wait_limit);
-    // shared memory: the query block, the key and value rings, P, barriers
+    // shared memory: the query block, the key ring, the value ring, P,
+    // barriers; two stages per ring where they fit, else one
     p.k_stage_bytes = kKeys * p.Dk * 2;
     p.v_stage_bytes = kKeys * p.Dv * 2;
     const int q_bytes = kRows * p.Dk * 2;
     const int p_bytes = kRows * kKeys * 2;
     const int fixed = q_bytes + p_bytes + static_cast<int>(sizeof(AttnBarriers)) + 64 + 1024;
-    p.stages = fixed + kMaxStages * (p.k_stage_bytes + p.v_stage_bytes) <= kSmemLimit ? kMaxStages : 1;
-    if (fixed + p.stages * (p.k_stage_bytes + p.v_stage_bytes) > kSmemLimit)
+    static const int kChoices[4][2] = {{2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    p.k_stages = 0;
+    for (const auto &c : kChoices)
+        if (fixed + c[0] * p.k_stage_bytes + c[1] * p.v_stage_bytes <= kSmemLimit) {
+            p.k_stages = c[0];
+            p.v_stages = c[1];
+            break;
+        }
+    if (p.k_stages == 0)
         return CSA_ERR_UNSUPPORTED;
     p.off_q = 0;
     p.off_k = q_bytes;
-    p.off_v = p.off_k + p.stages * p.k_stage_bytes;
-    p.off_p = p.off_v + p.stages * p.v_stage_bytes;
+    p.off_v = p.off_k + p.k_stages * p.k_stage_bytes;
+    p.off_p = p.off_v + p.v_stages * p.v_stage_bytes;
     p.off_bar = p.off_p + p_bytes;
     int smem_bytes = p.off_bar + static_cast<int>(sizeof(AttnBarriers)) + 64 + 1024;
     // more than half of the SM: one CTA per SM, so its 512-column TMEM
@@ -730,14 +738,20 @@ extern "C" csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaSt
     if (smem_bytes < kSmemLimit / 2 + 1024)
         smem_bytes = kSmemLimit / 2 + 1024;
 
-    CUtensorMap tmQ, tmK, tmV;
+    p.k = static_cast<const uint8_t *>(args->k);
+    p.v = static_cast<const uint8_t *>(args->v);
+    p.v_row_bytes = args->ld_v * 2;
+    CUtensorMap tmQ;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_tmap(&tmQ, bf, args->q, rows * p.HA, p.Dk, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap(&tmK, bf, args->k, static_cast<long long>(p.B) * p.T, p.Dk, 64, 1,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap(&tmV, bf, args->v, static_cast<long long>(p.B) * p.T, p.Dv, 64, 1,
-                   CU_TENSOR_MAP_SWIZZLE_128B, 2, args->ld_v))
+    if (!make_tmap(&tmQ, bf, args->q, rows * p.HA, p.Dk, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
         return CSA_ERR_CUDA;
+    // the warpgroups trade registers (setmaxnreg): only valid for a build
+    // with exactly the launch count the split assumes
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, sparse_attn_kernel) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    if (fa.numRegs != kLaunchRegs)
+        return CSA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_bytes) != cudaSuccess)
         return CSA_ERR_CUDA;
@@ -747,7 +761,7 @@ extern "C" csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaSt
     const int grid = rows < sms ? static_cast<int>(rows) : sms;
     if (!mark(0, stream))
         return CSA_ERR_CUDA;
-    sparse_attn_kernel<<<grid, kThreads, smem_bytes, stream>>>(tmQ, tmK, tmV, p);
+    sparse_attn_kernel<<<grid, kThreads, smem_bytes, stream>>>(tmQ, p);
     if (cudaGetLastError() != cudaSuccess)
         return CSA_ERR_CUDA;
     if (!mark(1, stream))

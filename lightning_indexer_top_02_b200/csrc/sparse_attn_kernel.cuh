@@ -4,19 +4,26 @@
 // per query, and a sparse attention kernel reads only those).
 //
 // For every query row (b, i) and head g < HA:
-//   J     = the selected keys idx[b,i,0..topk) (the indexer lists them first
-//           and pads with -1; entries outside [0, T) are ignored)
+//   J     = the entries of idx[b,i,0..topk) in [0, T), in slot order (the
+//           indexer lists its selection first and pads with -1; any entry
+//           outside [0, T) is padding, wherever it stands)
 //   o[g]  = softmax_j( scale * qa[g] . kc[J_j] ) . vc[J_j]     (0 if J is empty)
 // with one compressed cache row per key shared by every head; the value row
 // of key s is read from vc + (b*T + s) * ld_v, so values may be a prefix of
 // each key row (a latent cache) or a separate array.
 //
-// One persistent CTA per SM walks query rows.  Per row the selected keys go
-// through in tiles of 128:
-//   warp 4 (producer): the row's query block [128 head rows x Dk] by TMA, and
-//     per tile the 128 selected key rows and value rows by TMA gather (four
-//     rows per instruction) into a two-stage ring;
-//   warp 5 (MMA issuer, one thread; owns the TMEM allocation):
+// One persistent CTA per SM walks query rows.  Per row the slots up to the
+// last one that holds a key go through in tiles of 128:
+//   warp 9 (control): scans each row's index slots ahead of the others and
+//     publishes its tile count through a two-entry ring; loads the row's
+//     query block [128 head rows x Dk] by TMA;
+//   warps 4-7 (gather, 32 tile rows each, one per SM sub-partition): per tile
+//     the selected key rows and
+//     value rows by cp.async, 16 bytes per thread, written straight into the
+//     128-byte-swizzled K-major layout, into separate key and value rings (a
+//     key stage frees as soon as its S is computed); every thread's arrival
+//     on the stage's barrier fires when its copies have landed;
+//   warp 8 (MMA issuer, one thread; owns the TMEM allocation):
 //     S(t) = Q . K(t)^T into one of two 128-column TMEM slots (M = 128 head
 //     rows, N = 128 keys), then, once the softmax has written P(t-1),
 //     O += P(t-1) . V(t-1) into TMEM columns 256.. (N = Dv, V as an MN-major
@@ -25,8 +32,12 @@
 //     the row's tiles in the exp2 domain with the running maximum raised only
 //     when a tile exceeds it by more than 2^8 (then O is rescaled in TMEM),
 //     P in bf16 written to shared memory as the next MMA's K-major A
-//     operand, and at the end O / l to global memory (fp32).
-// Head rows past HA are computed and discarded (the MMA's M is 128).
+//     operand, and at the end O / l to global memory (fp32).  The tile's slot
+//     validity comes from index loads issued one tile ahead.
+// Head rows past HA are computed by the MMA and discarded; a softmax warp
+// whose 32 rows are all past HA only keeps the barrier protocol.  Warps 10-11
+// only complete the third warpgroup; registers move to the softmax
+// warpgroup (setmaxnreg).
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -40,18 +51,33 @@ namespace attn {
 
 constexpr int kKeys = 128;      // selected keys per tile (S's N, P.V's K)
 constexpr int kRows = 128;      // MMA M: head rows
-constexpr int kThreads = 192;   // warps 0-3 softmax, 4 producer, 5 MMA
-constexpr int kMaxStages = 2;
+constexpr int kThreads = 384;   // warps 0-3 softmax, 4-7 gather, 8 MMA, 9 control
+constexpr int kGatherWarps = 4;
+constexpr int kGatherRows = kKeys / kGatherWarps;   // tile rows per gather warp
+constexpr int kMmaWarp = 4 + kGatherWarps, kControlWarp = kMmaWarp + 1;
+// register split (setmaxnreg): launched with kLaunchRegs per thread, the
+// softmax warpgroup takes kSoftmaxRegs, the gather warpgroup kGatherRegs and
+// the MMA / control warpgroup kCtlRegs
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 240, kGatherRegs = 128, kCtlRegs = 136;
+static_assert(128 * (kSoftmaxRegs + kGatherRegs + kCtlRegs) == kThreads * kLaunchRegs,
+              "the register split must add up to the launch's registers");
+static_assert(kGatherRows == 32, "one index slot per gather lane");
+constexpr int kMaxStages = 2;   // per ring (keys, values)
 constexpr int kOCol = 256;      // first TMEM column of O (S slots take 0..255)
+constexpr int kScanChunk = 256; // index slots the producer scans per step (8 per lane)
 constexpr float kRescaleLog2 = 8.0f; // raise the running max only past 2^8
 
-enum Role : int { kRoleProducer = 21, kRoleMma = 22, kRoleSoftmax = 23 };
+enum Role : int { kRoleProducer = 21, kRoleMma = 22, kRoleSoftmax = 23, kRoleGather = 24 };
 
 struct AttnParams {
     int B, S, T, HA, Dk, Dv, topk;
-    int stages;
+    int k_stages, v_stages;
     float sl2;              // scale * log2(e)
     const int32_t *idx;     // [B*S, topk]
+    const uint8_t *k;       // key rows, Dk bf16 each
+    const uint8_t *v;       // value rows, ld_v bf16 apart
+    long long v_row_bytes;  // ld_v * 2
     float *out;             // [B*S, HA, Dv]
     int off_q, off_k, off_v, off_p, off_bar;   // shared-memory carve-up
     int k_stage_bytes, v_stage_bytes;
@@ -60,106 +86,200 @@ struct AttnParams {
 
 struct AttnBarriers {
     uint64_t q_full, q_empty;
-    uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
+    uint64_t k_full[kMaxStages], k_empty[kMaxStages];
+    uint64_t v_full[kMaxStages], v_empty[kMaxStages];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full, pv_done, o_empty;
+    uint64_t row_full[2], row_empty[2];
     uint64_t drain;
+    int row_tiles[2];       // tile count of the row published in each ring entry
+    int gather_rows[kGatherWarps][kGatherRows];   // global key rows of the tile, per gather warp
     uint32_t tmem_addr;
     int abort;
 };
 
 __device__ __forceinline__ bool key_ok(int32_t s, int T) { return s >= 0 && s < T; }
 
-// Selected keys of a query row: the indexer lists them first and pads with
-// -1, so the count is the first slot that holds no key (a full row is
-// recognised by its last slot; otherwise a bisection on that prefix).
-__device__ __forceinline__ int selected_count(const int32_t *row, int topk, int T)
+// Index slots base + 32u + lane (u < 8) of a row, -1 past topk.
+__device__ __forceinline__ void scan_load(const int32_t *row, int base, int topk, int lane,
+                                          int32_t (&v)[8])
 {
-    if (key_ok(__ldg(row + topk - 1), T))
-        return topk;
-    int lo = 0, hi = topk - 1;        // row[hi] holds no key
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (key_ok(__ldg(row + mid), T))
-            lo = mid + 1;
-        else
-            hi = mid;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int slot = base + 32 * u + lane;
+        v[u] = slot < topk ? __ldg(row + slot) : -1;
     }
-    return lo;
 }
 
-// ------------------------------------------------------------------ producer
-__device__ void attn_producer(const AttnParams &p, const CUtensorMap *tmQ, const CUtensorMap *tmK,
-                              const CUtensorMap *tmV, uint8_t *smem, AttnBarriers *bars,
-                              const WaitCtl &ctl)
+// The last slot of the chunk that holds a key, or -1 (warp-uniform).
+__device__ __forceinline__ int scan_last(const int32_t (&v)[8], int base, int T)
+{
+    int last = -1;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t b = __ballot_sync(0xffffffffu, key_ok(v[u], T));
+        if (b)
+            last = base + 32 * u + 31 - __clz(b);
+    }
+    return last;
+}
+
+// ------------------------------------------------------------------ control
+__device__ void attn_control(const AttnParams &p, const CUtensorMap *tmQ, uint8_t *smem,
+                             AttnBarriers *bars, const WaitCtl &ctl)
 {
     const int lane = threadIdx.x & 31;
-    int gt = 0, rows_used = 0;
-    const uint32_t kv_bytes = static_cast<uint32_t>(p.k_stage_bytes + p.v_stage_bytes);
+    const int rows = p.B * p.S;
+    int rows_used = 0;
     const uint32_t q_bytes = static_cast<uint32_t>(kRows * p.Dk * 2);
-    bool ok = true;
-    for (int r = blockIdx.x; r < p.B * p.S && ok; r += gridDim.x) {
+    // tile count of row r: the slots up to the last one that holds a key
+    auto row_tiles = [&](int r) -> int {
         const int32_t *row = p.idx + static_cast<size_t>(r) * p.topk;
-        const int n = selected_count(row, p.topk, p.T);
-        const int ntiles = (n + kKeys - 1) / kKeys;
-        if (ntiles == 0)
-            continue;
-        const int b = r / p.S;
-        // the query block: rows r*HA .. r*HA+127 of [B*S*HA, Dk] (padding head
-        // rows read the next rows or the zero fill past the end)
+        int last = -1;
+        for (int base = 0; base < p.topk; base += 2 * kScanChunk) {
+            int32_t v0[8], v1[8];
+            scan_load(row, base, p.topk, lane, v0);
+            scan_load(row, base + kScanChunk, p.topk, lane, v1);
+            last = max(last, scan_last(v0, base, p.T));
+            last = max(last, scan_last(v1, base + kScanChunk, p.T));
+        }
+        return (last + kKeys) / kKeys;
+    };
+    // publishes the tile count of the CTA's i-th row
+    auto publish = [&](int i, int nt) -> bool {
+        bool good = true;
         if (lane == 0) {
-            ok = wait_bounded(&bars->q_empty, (rows_used & 1) ^ 1, ctl, kRoleProducer, r);
-            if (ok) {
-                mbar_arrive_expect_tx(&bars->q_full, q_bytes);
-                for (int c = 0; c < p.Dk / 64; ++c)
-                    tma_load_2d(smem + p.off_q + c * kRows * 128, tmQ, &bars->q_full, 64 * c,
-                                r * p.HA);
+            good = wait_bounded(&bars->row_empty[i & 1], ((i >> 1) & 1) ^ 1, ctl, kRoleProducer, i);
+            if (good) {
+                bars->row_tiles[i & 1] = nt;
+                mbar_arrive(&bars->row_full[i & 1]);    // release: the count is visible
             }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok)
-            break;
-        ++rows_used;
-        for (int t = 0; t < ntiles && ok; ++t, ++gt) {
-            const int stage = gt % p.stages;
+        return __shfl_sync(0xffffffffu, good, 0);
+    };
+    int r = blockIdx.x;
+    int nt = row_tiles(r);
+    bool ok = publish(0, nt);
+    for (int i = 0; r < rows && ok; r += gridDim.x, ++i) {
+        if (nt > 0) {
+            // the query block: rows r*HA .. r*HA+127 of [B*S*HA, Dk] (padding
+            // head rows read the next rows or the zero fill past the end)
             if (lane == 0) {
-                ok = wait_bounded(&bars->kv_empty[stage], ((gt / p.stages) & 1) ^ 1, ctl,
-                                  kRoleProducer, r);
-                if (ok)
-                    mbar_arrive_expect_tx(&bars->kv_full[stage], kv_bytes);
+                ok = wait_bounded(&bars->q_empty, (rows_used & 1) ^ 1, ctl, kRoleProducer, r);
+                if (ok) {
+                    mbar_arrive_expect_tx(&bars->q_full, q_bytes);
+                    for (int c = 0; c < p.Dk / 64; ++c)
+                        tma_load_2d(smem + p.off_q + c * kRows * 128, tmQ, &bars->q_full, 64 * c,
+                                    r * p.HA);
+                }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok)
                 break;
-            // lane l gathers keys 4l .. 4l+3 of the tile; slots holding no key
-            // read row 0 of the batch (their scores are masked)
-            int rr[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int slot = t * kKeys + 4 * lane + e;
-                const int32_t s = slot < p.topk ? __ldg(row + slot) : -1;
-                rr[e] = b * p.T + (key_ok(s, p.T) ? s : 0);
-            }
-            uint8_t *kdst = smem + p.off_k + stage * p.k_stage_bytes + 4 * lane * 128;
-            uint8_t *vdst = smem + p.off_v + stage * p.v_stage_bytes + 4 * lane * 128;
-            for (int c = 0; c < p.Dk / 64; ++c)
-                tma_gather4(kdst + c * kKeys * 128, tmK, &bars->kv_full[stage], 64 * c, rr[0],
-                            rr[1], rr[2], rr[3]);
-            for (int c = 0; c < p.Dv / 64; ++c)
-                tma_gather4(vdst + c * kKeys * 128, tmV, &bars->kv_full[stage], 64 * c, rr[0],
-                            rr[1], rr[2], rr[3]);
+            ++rows_used;
+        }
+        const int rn = r + gridDim.x;
+        if (rn >= rows)
+            break;
+        nt = row_tiles(rn);
+        ok = publish(i + 1, nt);
+    }
+    // the query copies issued land before the CTA can exit
+    if (lane == 0 && rows_used > 0)
+        wait_drain(&bars->q_full, (rows_used - 1) & 1);
+}
+
+// ------------------------------------------------------------------ gather
+// Tile rows row0 .. row0+nrows-1 of one ring stage from global rows
+// grows[k] (row_bytes apart; 16-byte units, `units` per row), in the
+// 128-byte-swizzled K-major layout: 64-element chunk c of tile row k at
+// stage + c*128*128 + k*128, 16-byte unit u of the chunk at (u ^ (k & 7))*16.
+// Lane l copies unit q = l % units of rows k = l / units, + rpi, ...
+__device__ __forceinline__ void gather_stage(uint32_t stage, const uint8_t *base, long long row_bytes,
+                                             const int *grows, int row0, int nrows, int q, int k0,
+                                             int rpi)
+{
+    const int c = q >> 3, u = q & 7;
+    const uint32_t dst0 = stage + c * kRows * 128;
+    for (int k = k0; k < nrows; k += rpi) {
+        const int row = row0 + k;
+        cp_async_16(dst0 + row * 128 + ((u ^ (row & 7)) << 4),
+                    base + grows[k] * row_bytes + q * 16);
+    }
+}
+
+__device__ void attn_gather(const AttnParams &p, uint8_t *smem, AttnBarriers *bars, const WaitCtl &ctl)
+{
+    const int lane = threadIdx.x & 31;
+    const int gw = (threadIdx.x >> 5) - 4;        // gather warp 0 .. kGatherWarps-1
+    const int row0 = gw * kGatherRows;            // its rows of every tile
+    const int rows = p.B * p.S;
+    int *grows = bars->gather_rows[gw];
+    const uint32_t k_base = smem_u32(smem + p.off_k);
+    const uint32_t v_base = smem_u32(smem + p.off_v);
+    // lane -> (unit, first row, rows per instruction) for each operand width
+    const int ku = p.Dk / 8, vu = p.Dv / 8;
+    const int k_rpi = ku >= 32 ? 1 : 32 / ku, v_rpi = vu >= 32 ? 1 : 32 / vu;
+    const int k_q = lane % ku, v_q = lane % vu;
+    const int k_k0 = lane < k_rpi * ku ? lane / ku : kGatherRows;   // idle lanes copy nothing
+    const int v_k0 = lane < v_rpi * vu ? lane / vu : kGatherRows;
+    int gt = 0;
+    bool ok = true;
+    int32_t pf = -1;                              // the next tile's slot row0 + lane
+    auto prefetch = [&](int r, int t) {
+        const int slot = t * kKeys + row0 + lane;
+        pf = slot < p.topk ? __ldg(p.idx + static_cast<size_t>(r) * p.topk + slot) : -1;
+    };
+    prefetch(blockIdx.x, 0);
+    for (int r = blockIdx.x, i = 0; r < rows && ok; r += gridDim.x, ++i) {
+        int nt = 0;
+        if (lane == 0) {
+            ok = wait_bounded(&bars->row_full[i & 1], (i >> 1) & 1, ctl, kRoleGather, r);
+            if (ok)
+                nt = *reinterpret_cast<volatile int *>(&bars->row_tiles[i & 1]);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        nt = __shfl_sync(0xffffffffu, nt, 0);
+        if (!ok)
+            break;
+        if (lane == 0)
+            mbar_arrive(&bars->row_empty[i & 1]);
+        const int rn = r + gridDim.x;
+        const int bT = (r / p.S) * p.T;
+        if (nt == 0 && rn < rows)
+            prefetch(rn, 0);
+        for (int t = 0; t < nt; ++t, ++gt) {
+            // this tile's global key rows (slots holding no key read row 0 of
+            // the batch: their scores are masked)
+            __syncwarp();                         // the previous tile's copies have read grows
+            grows[lane] = bT + (key_ok(pf, p.T) ? pf : 0);
+            if (t + 1 < nt)
+                prefetch(r, t + 1);
+            else if (rn < rows)
+                prefetch(rn, 0);
+            __syncwarp();
+            const int ks = gt % p.k_stages, vs = gt % p.v_stages;
+            if (lane == 0)
+                ok = wait_bounded(&bars->k_empty[ks], ((gt / p.k_stages) & 1) ^ 1, ctl, kRoleGather, r);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok)
+                break;
+            gather_stage(k_base + ks * p.k_stage_bytes, p.k, static_cast<long long>(p.Dk) * 2, grows,
+                         row0, kGatherRows, k_q, k_k0, k_rpi);
+            cp_async_arrive_noinc(&bars->k_full[ks]);
+            if (lane == 0)
+                ok = wait_bounded(&bars->v_empty[vs], ((gt / p.v_stages) & 1) ^ 1, ctl, kRoleGather, r);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok)
+                break;
+            gather_stage(v_base + vs * p.v_stage_bytes, p.v, p.v_row_bytes, grows, row0, kGatherRows,
+                         v_q, v_k0, v_rpi);
+            cp_async_arrive_noinc(&bars->v_full[vs]);
         }
     }
-    // every copy issued lands before the CTA can exit
-    if (lane == 0) {
-        for (int s = 0; s < p.stages; ++s)
-            if (gt > s) {
-                const int fills = (gt - s + p.stages - 1) / p.stages;
-                wait_drain(&bars->kv_full[s], (fills - 1) & 1);
-            }
-        if (rows_used > 0)
-            wait_drain(&bars->q_full, (rows_used - 1) & 1);
-    }
+    if (!ok)
+        *ctl.abort = 1;
+    cp_async_wait_all();                          // every copy lands before the CTA can exit
 }
 
 // ------------------------------------------------------------------ MMA issuer
@@ -173,57 +293,60 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
     const uint32_t k_base = smem_u32(smem + p.off_k);
     const uint32_t v_base = smem_u32(smem + p.off_v);
     const uint32_t p_base = smem_u32(smem + p.off_p);
-    auto issue_pv = [&](int gu, bool first) -> bool {
-        if (!wait_bounded(&bars->p_full, gu & 1, ctl, kRoleMma, gu))
+    // O (+)= P(g) . V(g) for the CTA's g-th tile
+    auto issue_pv = [&](int g, bool first) -> bool {
+        const int vs = g % p.v_stages;
+        if (!wait_bounded(&bars->p_full, g & 1, ctl, kRoleMma, g) ||
+            !wait_bounded(&bars->v_full[vs], (g / p.v_stages) & 1, ctl, kRoleMma, g))
             return false;
         // the row's first P.V overwrites O: the previous row's O must have been read out
         if (first && rows_used > 0 &&
-            !wait_bounded(&bars->o_empty, (rows_used - 1) & 1, ctl, kRoleMma, gu))
+            !wait_bounded(&bars->o_empty, (rows_used - 1) & 1, ctl, kRoleMma, g))
             return false;
+        fence_proxy_async_smem();                    // cp.async (generic) writes -> tensor core reads
         tc_fence_after();
-        const int stage = gu % p.stages;
-        const uint32_t vst = v_base + stage * p.v_stage_bytes;
+        const uint32_t vst = v_base + vs * p.v_stage_bytes;
 #pragma unroll
         for (int ks = 0; ks < kKeys / 16; ++ks) {
             const uint64_t adesc = smem_desc_kmajor(p_base + (ks >> 2) * kRows * 128 + (ks & 3) * 32, 128);
             const uint64_t bdesc = smem_desc_mn_sw128(vst + ks * 16 * 128, kKeys * 128, 1024);
             mma_f16_ss(tmem + kOCol, adesc, bdesc, idesc_pv, (!first || ks > 0) ? 1u : 0u);
         }
-        mma_commit(&bars->kv_empty[stage]);
+        mma_commit(&bars->v_empty[vs]);
         mma_commit(&bars->pv_done);
         return true;
     };
     bool ok = true;
-    for (int r = blockIdx.x; r < p.B * p.S && ok; r += gridDim.x) {
-        const int32_t *row = p.idx + static_cast<size_t>(r) * p.topk;
-        const int n = selected_count(row, p.topk, p.T);
-        const int ntiles = (n + kKeys - 1) / kKeys;
-        if (ntiles == 0)
+    for (int r = blockIdx.x, i = 0; r < p.B * p.S && ok; r += gridDim.x, ++i) {
+        if (!wait_bounded(&bars->row_full[i & 1], (i >> 1) & 1, ctl, kRoleMma, r))
+            break;
+        const int nt = *reinterpret_cast<volatile int *>(&bars->row_tiles[i & 1]);
+        mbar_arrive(&bars->row_empty[i & 1]);
+        if (nt == 0)
             continue;
         if (!wait_bounded(&bars->q_full, rows_used & 1, ctl, kRoleMma, r))
             break;
         tc_fence_after();
         const int g0 = gt;
-        for (int t = 0; t < ntiles; ++t, ++gt) {
-            const int stage = gt % p.stages;
+        for (int t = 0; t < nt; ++t, ++gt) {
+            const int ks = gt % p.k_stages;
             const int slot = gt & 1;
-            // one stage: tile t's keys replace tile t-1's values, so P.V of
-            // tile t-1 goes first; with two, S(t) overlaps the softmax of t-1
-            if (p.stages == 1 && t > 0 && !(ok = issue_pv(gt - 1, gt - 1 == g0)))
-                break;
-            ok = wait_bounded(&bars->kv_full[stage], (gt / p.stages) & 1, ctl, kRoleMma, r) &&
+            ok = wait_bounded(&bars->k_full[ks], (gt / p.k_stages) & 1, ctl, kRoleMma, r) &&
                  wait_bounded(&bars->s_empty[slot], ((gt >> 1) & 1) ^ 1, ctl, kRoleMma, r);
             if (!ok)
                 break;
+            fence_proxy_async_smem();                // cp.async (generic) writes -> tensor core reads
             tc_fence_after();
-            const uint32_t kst = k_base + stage * p.k_stage_bytes;
-            for (int ks = 0; ks < p.Dk / 16; ++ks) {
-                const uint32_t co = (ks >> 2) * kRows * 128 + (ks & 3) * 32;
+            const uint32_t kst = k_base + ks * p.k_stage_bytes;
+            for (int kk = 0; kk < p.Dk / 16; ++kk) {
+                const uint32_t co = (kk >> 2) * kRows * 128 + (kk & 3) * 32;
                 mma_f16_ss(tmem + slot * kKeys, smem_desc_kmajor(q_base + co, 128),
-                           smem_desc_kmajor(kst + co, 128), idesc_s, ks > 0 ? 1u : 0u);
+                           smem_desc_kmajor(kst + co, 128), idesc_s, kk > 0 ? 1u : 0u);
             }
             mma_commit(&bars->s_full[slot]);
-            if (p.stages > 1 && t > 0 && !(ok = issue_pv(gt - 1, gt - 1 == g0)))
+            mma_commit(&bars->k_empty[ks]);
+            // S(t) is queued: P(t-1) . V(t-1) overlaps the softmax of tile t
+            if (t > 0 && !(ok = issue_pv(gt - 1, gt - 1 == g0)))
                 break;
         }
         if (!ok)
@@ -237,16 +360,84 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
 }
 
 // ------------------------------------------------------------------ softmax
-// Validity of the tile's 128 key slots as four 32-bit masks (bit j of mask w
-// = slot 32w + j), formed by each warp from the index row.
-__device__ __forceinline__ void tile_masks(const int32_t *row, int topk, int n, int T, int t,
-                                           int lane, uint32_t (&mask)[4])
+// The running maximum (log2 domain) after one tile of this thread's head row:
+// v = the row's 128 raw scores (TMEM image), mask = slot validity (bit j of
+// word w = slot 32w + j).  Returns the maximum to use and sets alpha, the
+// factor O and l must be scaled by (1 when the maximum was kept).
+template <bool kMasked>
+__device__ __forceinline__ float tile_max(const uint32_t (&v)[kKeys], const uint32_t (&mask)[4],
+                                          float sl2, float m, float &alpha)
 {
+    // extreme raw score in the direction of the scale's sign (NaN = masked,
+    // which fmaxf / fminf skip)
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        a[k] = kMasked ? NAN : __uint_as_float(v[k]);
+    const bool up = sl2 >= 0.0f;
+#pragma unroll
+    for (int j = kMasked ? 0 : 8; j < kKeys; ++j) {
+        float x = __uint_as_float(v[j]);
+        if (kMasked && !((mask[j >> 5] >> (j & 31)) & 1u))
+            x = NAN;
+        a[j & 7] = up ? fmaxf(a[j & 7], x) : fminf(a[j & 7], x);
+    }
+#pragma unroll
+    for (int k = 1; k < 8; ++k)
+        a[0] = up ? fmaxf(a[0], a[k]) : fminf(a[0], a[k]);
+    const float mt = a[0] == a[0] ? a[0] * sl2 : -INFINITY;
+    alpha = 1.0f;
+    if (m == -INFINITY)
+        return mt;                                   // first keys of the row
+    if (mt > m + kRescaleLog2) {
+        alpha = ex2_approx(m - mt);
+        return mt;
+    }
+    return m;
+}
+
+// P for one tile: p_j = 2^(sl2 * v_j - m) (0 for masked slots), rounded to
+// bf16 and stored as the row's 128 keys of the K-major A operand (two
+// 64-key chunks of 128-byte rows, 16-byte units swizzled by the row's low 3
+// bits); returns the tile's sum of p (fp32).
+template <bool kMasked>
+__device__ __forceinline__ float tile_probs(const uint32_t (&v)[kKeys], const uint32_t (&mask)[4],
+                                            float sl2, float m, uint8_t *pbuf, int hrow)
+{
+    float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const float nm = -m;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int j = 8 * u + 2 * h;
+            float p0 = ex2_approx(fmaf(__uint_as_float(v[j]), sl2, nm));
+            float p1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), sl2, nm));
+            if (kMasked) {
+                p0 = ((mask[j >> 5] >> (j & 31)) & 1u) ? p0 : 0.0f;
+                p1 = ((mask[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u) ? p1 : 0.0f;
+            }
+            s[h] += p0 + p1;
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            w[h] = *reinterpret_cast<const uint32_t *>(&b2);
+        }
+        const int c = u >> 3, uu = u & 7;
+        *reinterpret_cast<uint4 *>(pbuf + c * kRows * 128 + hrow * 128 + ((uu ^ (hrow & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return (s[0] + s[1]) + (s[2] + s[3]);
+}
+
+// Index slots 32w + lane (w < 4) of tile t of row r, -1 past topk.
+__device__ __forceinline__ void mask_slots(const AttnParams &p, int r, int t, int lane,
+                                           int32_t (&v)[4])
+{
+    const int32_t *row = p.idx + static_cast<size_t>(r) * p.topk;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
         const int slot = t * kKeys + 32 * w + lane;
-        const bool ok = slot < n && key_ok(__ldg(row + slot), T);
-        mask[w] = __ballot_sync(0xffffffffu, ok);
+        v[w] = slot < p.topk ? __ldg(row + slot) : -1;
     }
 }
 
@@ -256,104 +447,117 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int hrow = threadIdx.x;                 // head row = TMEM lane
+    const bool active = warp * 32 < p.HA;         // the warp's rows include heads
+    const int rows = p.B * p.S;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     uint8_t *pbuf = smem + p.off_p;
-    int gt = 0, rows_used = 0;
+    int gt = 0;
     bool ok = true;
-    for (int r = blockIdx.x; r < p.B * p.S && ok; r += gridDim.x) {
-        const int32_t *row = p.idx + static_cast<size_t>(r) * p.topk;
-        const int n = selected_count(row, p.topk, p.T);
-        const int ntiles = (n + kKeys - 1) / kKeys;
+    int32_t pf[4] = {-1, -1, -1, -1};             // the next tile's index slots, in flight
+    if (active)
+        mask_slots(p, blockIdx.x, 0, lane, pf);
+    for (int r = blockIdx.x, i = 0; r < rows && ok; r += gridDim.x, ++i) {
+        int nt = 0;
+        if (lane == 0) {
+            ok = wait_bounded(&bars->row_full[i & 1], (i >> 1) & 1, ctl, kRoleSoftmax, r);
+            if (ok)
+                nt = *reinterpret_cast<volatile int *>(&bars->row_tiles[i & 1]);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        nt = __shfl_sync(0xffffffffu, nt, 0);
+        if (!ok)
+            break;
+        if (lane == 0)
+            mbar_arrive(&bars->row_empty[i & 1]);
+        const int rn = r + gridDim.x;
         float *orow = p.out + (static_cast<size_t>(r) * p.HA + hrow) * p.Dv;
-        if (ntiles == 0) {
+        if (nt == 0) {
             if (hrow < p.HA)
                 for (int e = 0; e < p.Dv; e += 4)
                     *reinterpret_cast<float4 *>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (active && rn < rows)
+                mask_slots(p, rn, 0, lane, pf);
             continue;
         }
         float m = -INFINITY, l = 0.0f;
-        for (int t = 0; t < ntiles; ++t, ++gt) {
+        for (int t = 0; t < nt; ++t, ++gt) {
             const int slot = gt & 1;
-            uint32_t mask[4];
-            tile_masks(row, p.topk, n, p.T, t, lane, mask);
+            uint32_t mask[4] = {0u, 0u, 0u, 0u};
+            if (active) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    mask[w] = __ballot_sync(0xffffffffu, key_ok(pf[w], p.T));
+                if (t + 1 < nt)
+                    mask_slots(p, r, t + 1, lane, pf);
+                else if (rn < rows)
+                    mask_slots(p, rn, 0, lane, pf);
+            }
             ok = wait_bounded(&bars->s_full[slot], (gt >> 1) & 1, ctl, kRoleSoftmax, r);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 break;
             tc_fence_after();
-            float x[kKeys];
-            {
-                uint32_t v[32];
+            if (active) {
+                uint32_t v[kKeys];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld_32x32b_x32(lane_base + slot * kKeys + 32 * c, v);
-                    tmem_ld_wait();
+                for (int c = 0; c < 4; ++c)
+                    tmem_ld_32x32b_x32(lane_base + slot * kKeys + 32 * c,
+                                       *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+                tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[32 * c + j] = ((mask[c] >> j) & 1u) ? __uint_as_float(v[j]) * p.sl2
-                                                              : -INFINITY;
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars->s_empty[slot]);     // the S slot may be overwritten
-            float mt = -INFINITY;
+                for (int j = 0; j < kKeys; ++j)
+                    reg_fence(v[j]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->s_empty[slot]);     // the S slot may be overwritten
+                const bool full = (mask[0] & mask[1] & mask[2] & mask[3]) == 0xFFFFFFFFu;
+                float alpha;
+                const float m_new = full ? tile_max<false>(v, mask, p.sl2, m, alpha)
+                                         : tile_max<true>(v, mask, p.sl2, m, alpha);
+                // the previous tile's P.V is done: P may be overwritten and O is stable
+                if (t > 0) {
+                    ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+                        // O (TMEM, this thread's row) *= alpha, 32 columns at a time
+                        for (int c = 0; c < p.Dv / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld_32x32b_x32(lane_base + kOCol + 32 * c, o);
+                            tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < kKeys; ++j)
-                mt = fmaxf(mt, x[j]);
-            float m_use = m, alpha = 1.0f;
-            bool rescale = false;
-            if (m == -INFINITY) {
-                m_use = mt;                            // first keys of the row
-            } else if (mt > m + kRescaleLog2) {
-                m_use = mt;
-                alpha = exp2f(m - mt);
-                rescale = true;
-            }
-            float sum = 0.0f;
-            uint32_t pk[kKeys / 2];
-#pragma unroll
-            for (int j = 0; j < kKeys; j += 2) {
-                const float p0 = m_use == -INFINITY ? 0.0f : exp2f(x[j] - m_use);
-                const float p1 = m_use == -INFINITY ? 0.0f : exp2f(x[j + 1] - m_use);
-                sum += p0 + p1;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                pk[j / 2] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-            l = l * alpha + sum;
-            m = m_use;
-            // the previous tile's P.V is done: P may be overwritten and O is stable
-            if (t > 0) {
-                ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok)
-                    break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // O (TMEM, this thread's row) *= alpha, 32 columns at a time
-                    for (int c = 0; c < p.Dv / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(lane_base + kOCol + 32 * c, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-                        tmem_st_32x32b_x32(lane_base + kOCol + 32 * c, v);
+                            for (int j = 0; j < 32; ++j)
+                                o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st_32x32b_x32(lane_base + kOCol + 32 * c, o);
+                        }
+                        tmem_st_wait();
                     }
-                    tmem_st_wait();
+                }
+                float sum = 0.0f;
+                if (m_new != -INFINITY)
+                    sum = full ? tile_probs<false>(v, mask, p.sl2, m_new, pbuf, hrow)
+                               : tile_probs<true>(v, mask, p.sl2, m_new, pbuf, hrow);
+                else
+                    for (int u = 0; u < 16; ++u)         // no key yet: P = 0
+                        *reinterpret_cast<uint4 *>(pbuf + (u >> 3) * kRows * 128 + hrow * 128 +
+                                                   ((u & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                l = l * alpha + sum;
+                m = m_new;
+                fence_proxy_async_smem();
+            } else {
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->s_empty[slot]);
+                if (t > 0) {
+                    ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok)
+                        break;
                 }
             }
-            // P row: 128 bf16 keys as two 64-key chunks of the K-major operand
-            // (128-byte rows, 16-byte units swizzled by the row's low 3 bits)
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int c = u >> 3, uu = u & 7;
-                uint8_t *dst = pbuf + c * kRows * 128 + hrow * 128 + ((uu ^ (hrow & 7)) << 4);
-                *reinterpret_cast<uint4 *>(dst) =
-                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            }
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -367,24 +571,25 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
         if (!ok)
             break;
         tc_fence_after();
-        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-        for (int c = 0; c < p.Dv / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(lane_base + kOCol + 32 * c, v);
-            tmem_ld_wait();
-            if (hrow < p.HA) {
+        if (active) {
+            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+            for (int c = 0; c < p.Dv / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(lane_base + kOCol + 32 * c, o);
+                tmem_ld_wait();
+                if (hrow < p.HA) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(orow + 32 * c + j) =
-                        make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
-                                    __uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(orow + 32 * c + j) =
+                            make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
+                                        __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+                }
             }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&bars->o_empty);
-        ++rows_used;
     }
     if (!ok)
         *ctl.abort = 1;
@@ -392,8 +597,7 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
 
 // ------------------------------------------------------------------ kernel
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const AttnParams p)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const AttnParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -405,12 +609,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
+            mbar_init(&bars->k_full[s], kGatherWarps * 32);   // one arrival per gather thread
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], kGatherWarps * 32);
+            mbar_init(&bars->v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
             mbar_init(&bars->s_empty[s], 4);
+            mbar_init(&bars->row_full[s], 1);
+            mbar_init(&bars->row_empty[s], 5 + kGatherWarps);   // MMA, softmax and gather warps
         }
         mbar_init(&bars->p_full, 4);
         mbar_init(&bars->pv_done, 1);
@@ -419,10 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bars->abort = 0;
         fence_mbar_init();
         prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&bars->tmem_addr, 512);
         tmem_relinquish();
     }
@@ -431,16 +637,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_addr;
     WaitCtl ctl{&bars->abort, p.wait_limit};
-    if (warp < 4)
+    if (warp < 4) {
+        regs_inc<kSoftmaxRegs>();
         attn_softmax(p, smem, bars, tmem, ctl);
-    else if (warp == 4)
-        attn_producer(p, &tmQ, &tmK, &tmV, smem, bars, ctl);
-    else if (lane == 0)
-        attn_mma(p, smem, bars, tmem, ctl);
+    } else if (warp < 4 + kGatherWarps) {
+        regs_dec<kGatherRegs>();
+        attn_gather(p, smem, bars, ctl);
+    } else {
+        regs_dec<kCtlRegs>();
+        if (warp == kMmaWarp) {
+            if (lane == 0)
+                attn_mma(p, smem, bars, tmem, ctl);
+        } else if (warp == kControlWarp) {
+            attn_control(p, &tmQ, smem, bars, ctl);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         tmem_dealloc(tmem, 512);
     }

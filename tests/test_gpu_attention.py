@@ -92,15 +92,21 @@ def test_attention_full_topk_rows(lib):
 
 
 def test_attention_padding_and_empty_rows(lib):
-    """Rows with no selected key give zeros; padding slots are ignored."""
-    B, S, T, topk = 1, 6, 300, 130
+    """Rows with no selected key give zeros; padding slots (-1 or >= T) are
+    ignored wherever they stand, including between keys and in whole tiles."""
+    B, S, T, topk = 1, 8, 300, 390
     idx = torch.full((B, S, topk), -1, dtype=torch.int32, device="cuda")
     idx[0, 1, :1] = 17
     idx[0, 2, :129] = torch.arange(129, dtype=torch.int32, device="cuda")
     idx[0, 3, :130] = torch.arange(130, 260, dtype=torch.int32, device="cuda")
+    idx[0, 5, 0:390:3] = torch.arange(0, 260, 2, dtype=torch.int32, device="cuda")  # holes
+    idx[0, 5, 7] = T + 5                                                           # out of range
+    idx[0, 6, 300] = 42                                    # one key in the third tile only
+    idx[0, 7, 128:256] = torch.arange(128, dtype=torch.int32, device="cuda")       # empty first tile
     got, ref = attn_case(lib, B=B, S=S, T=T, HA=8, Dk=64, Dv=64, topk=topk, seed=9,
                          idx_override=idx)
     assert np.all(got[0] == 0.0) and np.all(got[4] == 0.0)
+    assert np.any(got[5] != 0.0) and np.any(got[6] != 0.0)
 
 
 def test_attention_large_logits_rescale(lib):
