@@ -743,7 +743,11 @@ extern "C" csa_status_t csa_sparse_attention(const csa_attn_args_t *args, cudaSt
     p.v_row_bytes = args->ld_v * 2;
     CUtensorMap tmQ;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_tmap(&tmQ, bf, args->q, rows * p.HA, p.Dk, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    // HA <= 64: the query block (64 rows) is loaded twice and the warp pairs
+    // split each tile's keys; otherwise one 128-row block
+    p.split = p.HA <= kRows / 2 ? 1 : 0;
+    if (!make_tmap(&tmQ, bf, args->q, rows * p.HA, p.Dk, 64, p.split ? kRows / 2 : kRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
         return CSA_ERR_CUDA;
     // the warpgroups trade registers (setmaxnreg): only valid for a build
     // with exactly the launch count the split assumes

@@ -14,16 +14,16 @@
 //
 // One persistent CTA per SM walks query rows.  Per row the slots up to the
 // last one that holds a key go through in tiles of 128:
-//   warp 9 (control): scans each row's index slots ahead of the others and
+//   warp 13 (control): scans each row's index slots ahead of the others and
 //     publishes its tile count through a two-entry ring; loads the row's
 //     query block [128 head rows x Dk] by TMA;
-//   warps 4-7 (gather, 32 tile rows each, one per SM sub-partition): per tile
-//     the selected key rows and
+//   warps 4-11 (gather, 16 tile rows each, two per SM sub-partition): per
+//     tile the selected key rows and
 //     value rows by cp.async, 16 bytes per thread, written straight into the
 //     128-byte-swizzled K-major layout, into separate key and value rings (a
 //     key stage frees as soon as its S is computed); every thread's arrival
 //     on the stage's barrier fires when its copies have landed;
-//   warp 8 (MMA issuer, one thread; owns the TMEM allocation):
+//   warp 12 (MMA issuer, one thread; owns the TMEM allocation):
 //     S(t) = Q . K(t)^T into one of two 128-column TMEM slots (M = 128 head
 //     rows, N = 128 keys), then, once the softmax has written P(t-1),
 //     O += P(t-1) . V(t-1) into TMEM columns 256.. (N = Dv, V as an MN-major
@@ -35,8 +35,8 @@
 //     operand, and at the end O / l to global memory (fp32).  The tile's slot
 //     validity comes from index loads issued one tile ahead.
 // Head rows past HA are computed by the MMA and discarded; a softmax warp
-// whose 32 rows are all past HA only keeps the barrier protocol.  Warps 10-11
-// only complete the third warpgroup; registers move to the softmax
+// whose 32 rows are all past HA only keeps the barrier protocol.  Warps 14-15
+// only complete the last warpgroup; registers move to the softmax
 // warpgroup (setmaxnreg).
 #pragma once
 #include <cuda.h>
@@ -51,18 +51,27 @@ namespace attn {
 
 constexpr int kKeys = 128;      // selected keys per tile (S's N, P.V's K)
 constexpr int kRows = 128;      // MMA M: head rows
-constexpr int kThreads = 384;   // warps 0-3 softmax, 4-7 gather, 8 MMA, 9 control
-constexpr int kGatherWarps = 4;
+constexpr int kThreads = 512;   // warps 0-3 softmax, 4-11 gather, 12 MMA, 13 control
+constexpr int kGatherWarps = 8;  // two warpgroups
 constexpr int kGatherRows = kKeys / kGatherWarps;   // tile rows per gather warp
 constexpr int kMmaWarp = 4 + kGatherWarps, kControlWarp = kMmaWarp + 1;
 // register split (setmaxnreg): launched with kLaunchRegs per thread, the
-// softmax warpgroup takes kSoftmaxRegs, the gather warpgroup kGatherRegs and
-// the MMA / control warpgroup kCtlRegs
-constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 240, kGatherRegs = 128, kCtlRegs = 136;
-static_assert(128 * (kSoftmaxRegs + kGatherRegs + kCtlRegs) == kThreads * kLaunchRegs,
-              "the register split must add up to the launch's registers");
-static_assert(kGatherRows == 32, "one index slot per gather lane");
+// softmax warpgroup raises its count to kSoftmaxRegs, each gather warpgroup
+// lowers its count to kGatherRegs, the MMA / control warpgroup keeps the
+// launch count.  An increase must not go below, a decrease not above, the
+// count a warpgroup holds, and the increase can only take what the decreases
+// released.
+constexpr int kLaunchRegs = 128;
+constexpr int kSoftmaxRegs = 248, kGatherRegs = 64;
+static_assert(kSoftmaxRegs >= kLaunchRegs && kGatherRegs <= kLaunchRegs &&
+                  kSoftmaxRegs % 8 == 0 && kGatherRegs % 8 == 0 && kSoftmaxRegs <= 256 &&
+                  kGatherRegs >= 24,
+              "setmaxnreg counts: increases from, decreases to at most, the launch count");
+static_assert(kSoftmaxRegs - kLaunchRegs <= 2 * (kLaunchRegs - kGatherRegs),
+              "the softmax increase must fit in what the gather warpgroups release");
+static_assert(128 * (kSoftmaxRegs + 2 * kGatherRegs + kLaunchRegs) <= kThreads * kLaunchRegs,
+              "the register split must fit in the launch's registers");
+static_assert(kGatherRows <= 32 && kGatherWarps % 4 == 0, "one index slot per gather lane");
 constexpr int kMaxStages = 2;   // per ring (keys, values)
 constexpr int kOCol = 256;      // first TMEM column of O (S slots take 0..255)
 constexpr int kScanChunk = 256; // index slots the producer scans per step (8 per lane)
@@ -73,6 +82,7 @@ enum Role : int { kRoleProducer = 21, kRoleMma = 22, kRoleSoftmax = 23, kRoleGat
 struct AttnParams {
     int B, S, T, HA, Dk, Dv, topk;
     int k_stages, v_stages;
+    int split;              // HA <= 64: each query block loaded twice, keys split over warp pairs
     float sl2;              // scale * log2(e)
     const int32_t *idx;     // [B*S, topk]
     const uint8_t *k;       // key rows, Dk bf16 each
@@ -94,6 +104,8 @@ struct AttnBarriers {
     uint64_t drain;
     int row_tiles[2];       // tile count of the row published in each ring entry
     int gather_rows[kGatherWarps][kGatherRows];   // global key rows of the tile, per gather warp
+    uint64_t xbar[2][2];    // split mode: per head-row pair, two exchange phases
+    float xchg[2][4][32];   // split mode: exchanged partial maxima / sums
     uint32_t tmem_addr;
     int abort;
 };
@@ -168,9 +180,11 @@ __device__ void attn_control(const AttnParams &p, const CUtensorMap *tmQ, uint8_
                 ok = wait_bounded(&bars->q_empty, (rows_used & 1) ^ 1, ctl, kRoleProducer, r);
                 if (ok) {
                     mbar_arrive_expect_tx(&bars->q_full, q_bytes);
+                    // split mode: a 64-row box, loaded into rows 0-63 and 64-127
                     for (int c = 0; c < p.Dk / 64; ++c)
-                        tma_load_2d(smem + p.off_q + c * kRows * 128, tmQ, &bars->q_full, 64 * c,
-                                    r * p.HA);
+                        for (int d = 0; d < (p.split ? 2 : 1); ++d)
+                            tma_load_2d(smem + p.off_q + c * kRows * 128 + d * 64 * 128, tmQ,
+                                        &bars->q_full, 64 * c, r * p.HA);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -228,7 +242,8 @@ __device__ void attn_gather(const AttnParams &p, uint8_t *smem, AttnBarriers *ba
     int32_t pf = -1;                              // the next tile's slot row0 + lane
     auto prefetch = [&](int r, int t) {
         const int slot = t * kKeys + row0 + lane;
-        pf = slot < p.topk ? __ldg(p.idx + static_cast<size_t>(r) * p.topk + slot) : -1;
+        pf = lane < kGatherRows && slot < p.topk
+                 ? __ldg(p.idx + static_cast<size_t>(r) * p.topk + slot) : -1;
     };
     prefetch(blockIdx.x, 0);
     for (int r = blockIdx.x, i = 0; r < rows && ok; r += gridDim.x, ++i) {
@@ -252,7 +267,8 @@ __device__ void attn_gather(const AttnParams &p, uint8_t *smem, AttnBarriers *ba
             // this tile's global key rows (slots holding no key read row 0 of
             // the batch: their scores are masked)
             __syncwarp();                         // the previous tile's copies have read grows
-            grows[lane] = bT + (key_ok(pf, p.T) ? pf : 0);
+            if (lane < kGatherRows)
+                grows[lane] = bT + (key_ok(pf, p.T) ? pf : 0);
             if (t + 1 < nt)
                 prefetch(r, t + 1);
             else if (rn < rows)
@@ -331,6 +347,15 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
         for (int t = 0; t < nt; ++t, ++gt) {
             const int ks = gt % p.k_stages;
             const int slot = gt & 1;
+            // P(t-1) already written while K(t) is still arriving: its P.V goes first
+            bool pv_pending = t > 0;
+            if (pv_pending && mbar_try_wait(&bars->p_full, (gt - 1) & 1, false) &&
+                mbar_try_wait(&bars->v_full[(gt - 1) % p.v_stages], ((gt - 1) / p.v_stages) & 1, false) &&
+                !mbar_try_wait(&bars->k_full[ks], (gt / p.k_stages) & 1, false)) {
+                if (!(ok = issue_pv(gt - 1, gt - 1 == g0)))
+                    break;
+                pv_pending = false;
+            }
             ok = wait_bounded(&bars->k_full[ks], (gt / p.k_stages) & 1, ctl, kRoleMma, r) &&
                  wait_bounded(&bars->s_empty[slot], ((gt >> 1) & 1) ^ 1, ctl, kRoleMma, r);
             if (!ok)
@@ -346,7 +371,7 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
             mma_commit(&bars->s_full[slot]);
             mma_commit(&bars->k_empty[ks]);
             // S(t) is queued: P(t-1) . V(t-1) overlaps the softmax of tile t
-            if (t > 0 && !(ok = issue_pv(gt - 1, gt - 1 == g0)))
+            if (pv_pending && !(ok = issue_pv(gt - 1, gt - 1 == g0)))
                 break;
         }
         if (!ok)
@@ -360,32 +385,46 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
 }
 
 // ------------------------------------------------------------------ softmax
-// The running maximum (log2 domain) after one tile of this thread's head row:
-// v = the row's 128 raw scores (TMEM image), mask = slot validity (bit j of
-// word w = slot 32w + j).  Returns the maximum to use and sets alpha, the
-// factor O and l must be scaled by (1 when the maximum was kept).
-template <bool kMasked>
-__device__ __forceinline__ float tile_max(const uint32_t (&v)[kKeys], const uint32_t (&mask)[4],
-                                          float sl2, float m, float &alpha)
+// Raw extreme of a thread's NC scores of the tile (v = TMEM image, mk = their
+// slot validity, bit j of word j/32): the maximum for a non-negative scale,
+// the minimum otherwise (the one that becomes the largest scale * s).
+// Masked slots are skipped; NaN when none is valid.
+template <bool kMasked, int NC>
+__device__ __forceinline__ float tile_extreme(const uint32_t (&v)[NC], const uint32_t (&mk)[NC / 32],
+                                              bool up)
 {
-    // extreme raw score in the direction of the scale's sign (NaN = masked,
-    // which fmaxf / fminf skip)
     float a[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
         a[k] = kMasked ? NAN : __uint_as_float(v[k]);
-    const bool up = sl2 >= 0.0f;
+    auto pick = [&](int j) -> float {
+        const float x = __uint_as_float(v[j]);
+        return kMasked && !((mk[j >> 5] >> (j & 31)) & 1u) ? NAN : x;
+    };
+    if (up) {
 #pragma unroll
-    for (int j = kMasked ? 0 : 8; j < kKeys; ++j) {
-        float x = __uint_as_float(v[j]);
-        if (kMasked && !((mask[j >> 5] >> (j & 31)) & 1u))
-            x = NAN;
-        a[j & 7] = up ? fmaxf(a[j & 7], x) : fminf(a[j & 7], x);
+        for (int j = kMasked ? 0 : 8; j < NC; ++j)
+            a[j & 7] = fmaxf(a[j & 7], pick(j));
+#pragma unroll
+        for (int k = 1; k < 8; ++k)
+            a[0] = fmaxf(a[0], a[k]);
+    } else {
+#pragma unroll
+        for (int j = kMasked ? 0 : 8; j < NC; ++j)
+            a[j & 7] = fminf(a[j & 7], pick(j));
+#pragma unroll
+        for (int k = 1; k < 8; ++k)
+            a[0] = fminf(a[0], a[k]);
     }
-#pragma unroll
-    for (int k = 1; k < 8; ++k)
-        a[0] = up ? fmaxf(a[0], a[k]) : fminf(a[0], a[k]);
-    const float mt = a[0] == a[0] ? a[0] * sl2 : -INFINITY;
+    return a[0];
+}
+
+// The running maximum (log2 domain) after a tile whose raw extreme is e: the
+// maximum is raised only when the tile exceeds it by more than 2^8; alpha is
+// the factor O and l must then be scaled by (1 when it was kept).
+__device__ __forceinline__ float next_max(float e, float sl2, float m, float &alpha)
+{
+    const float mt = e == e ? e * sl2 : -INFINITY;
     alpha = 1.0f;
     if (m == -INFINITY)
         return mt;                                   // first keys of the row
@@ -396,18 +435,21 @@ __device__ __forceinline__ float tile_max(const uint32_t (&v)[kKeys], const uint
     return m;
 }
 
-// P for one tile: p_j = 2^(sl2 * v_j - m) (0 for masked slots), rounded to
-// bf16 and stored as the row's 128 keys of the K-major A operand (two
-// 64-key chunks of 128-byte rows, 16-byte units swizzled by the row's low 3
-// bits); returns the tile's sum of p (fp32).
-template <bool kMasked>
-__device__ __forceinline__ float tile_probs(const uint32_t (&v)[kKeys], const uint32_t (&mask)[4],
-                                            float sl2, float m, uint8_t *pbuf, int hrow)
+// P for a thread's NC keys: p_j = 2^(sl2 * v_j - m) (0 for masked slots),
+// rounded to bf16 and stored as 16-byte units of the K-major A operand
+// (64-key chunks of 128-byte rows, unit u of row r at ((u ^ (r & 7)) * 16),
+// chunks kRows * 128 bytes apart): the thread's keys start at chunk c0 of
+// row r, and with kDup the same units also go to row r + 64.  Returns the
+// sum of the thread's p (fp32).
+template <bool kMasked, int NC, bool kDup>
+__device__ __forceinline__ float tile_probs(const uint32_t (&v)[NC], const uint32_t (&mk)[NC / 32],
+                                            float sl2, float m, uint8_t *pbuf, int r, int c0)
 {
     float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const float nm = -m;
+    uint8_t *row = pbuf + c0 * kRows * 128 + r * 128;
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
+    for (int u = 0; u < NC / 8; ++u) {
         uint32_t w[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
@@ -415,16 +457,17 @@ __device__ __forceinline__ float tile_probs(const uint32_t (&v)[kKeys], const ui
             float p0 = ex2_approx(fmaf(__uint_as_float(v[j]), sl2, nm));
             float p1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), sl2, nm));
             if (kMasked) {
-                p0 = ((mask[j >> 5] >> (j & 31)) & 1u) ? p0 : 0.0f;
-                p1 = ((mask[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u) ? p1 : 0.0f;
+                p0 = ((mk[j >> 5] >> (j & 31)) & 1u) ? p0 : 0.0f;
+                p1 = ((mk[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u) ? p1 : 0.0f;
             }
             s[h] += p0 + p1;
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
             w[h] = *reinterpret_cast<const uint32_t *>(&b2);
         }
-        const int c = u >> 3, uu = u & 7;
-        *reinterpret_cast<uint4 *>(pbuf + c * kRows * 128 + hrow * 128 + ((uu ^ (hrow & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        uint8_t *dst = row + (u >> 3) * kRows * 128 + (((u & 7) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (kDup)
+            *reinterpret_cast<uint4 *>(dst + 64 * 128) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     return (s[0] + s[1]) + (s[2] + s[3]);
 }
@@ -441,18 +484,46 @@ __device__ __forceinline__ void mask_slots(const AttnParams &p, int r, int t, in
     }
 }
 
+// Softmax warps.  Full mode (HA > 64): warp w owns head rows 32w.. (its TMEM
+// lane quarter) and all 128 keys of a tile.  Split mode (HA <= 64, the query
+// block loaded twice so that TMEM lanes 64-127 repeat rows 0-63): warps w and
+// w ^ 2 own the same 32 head rows, w the keys 64 * (w >> 1) .. +63 of every
+// tile and the columns Dv/2 * (w >> 1) .. of O; the pair exchanges its
+// partial row maxima per tile and its partial sums per row through shared
+// memory (bounded waits on a pair barrier), and P is written to both copies
+// of each row.
+template <bool kSplit>
 __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *bars, uint32_t tmem,
                              const WaitCtl &ctl)
 {
+    constexpr int NC = kSplit ? kKeys / 2 : kKeys;   // keys per thread per tile
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int hrow = threadIdx.x;                 // head row = TMEM lane
-    const bool active = warp * 32 < p.HA;         // the warp's rows include heads
+    const int q = kSplit ? (warp & 1) : warp;        // head-row quarter
+    const int half = kSplit ? (warp >> 1) : 0;       // key / output-column half
+    const int hrow = 32 * q + lane;                  // head row
+    const bool active = 32 * q < p.HA;               // the warp's rows include heads
     const int rows = p.B * p.S;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int o_cols = kSplit ? p.Dv / 2 : p.Dv;     // O columns this warp rescales and writes
+    const int o_col0 = half * o_cols;
+    const bool up = p.sl2 >= 0.0f;
     uint8_t *pbuf = smem + p.off_p;
-    int gt = 0;
+    int gt = 0, xc = 0;
     bool ok = true;
+    // pair exchange (split mode): write own value, arrive, wait for the partner's
+    auto exchange = [&](float mine) -> float {
+        float *buf = bars->xchg[xc & 1][warp];
+        buf[lane] = mine;
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&bars->xbar[q][xc & 1]);
+        const bool good = wait_bounded(&bars->xbar[q][xc & 1], (xc >> 1) & 1, ctl, kRoleSoftmax, xc);
+        ok = __all_sync(0xffffffffu, good);
+        const float other = bars->xchg[xc & 1][warp ^ 2][lane];
+        ++xc;
+        return other;
+    };
     int32_t pf[4] = {-1, -1, -1, -1};             // the next tile's index slots, in flight
     if (active)
         mask_slots(p, blockIdx.x, 0, lane, pf);
@@ -473,7 +544,7 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
         float *orow = p.out + (static_cast<size_t>(r) * p.HA + hrow) * p.Dv;
         if (nt == 0) {
             if (hrow < p.HA)
-                for (int e = 0; e < p.Dv; e += 4)
+                for (int e = o_col0; e < o_col0 + o_cols; e += 4)
                     *reinterpret_cast<float4 *>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
             if (active && rn < rows)
                 mask_slots(p, rn, 0, lane, pf);
@@ -498,23 +569,36 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
                 break;
             tc_fence_after();
             if (active) {
-                uint32_t v[kKeys];
+                uint32_t v[NC];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tmem_ld_32x32b_x32(lane_base + slot * kKeys + 32 * c,
+                for (int c = 0; c < NC / 32; ++c)
+                    tmem_ld_32x32b_x32(lane_base + slot * kKeys + half * NC + 32 * c,
                                        *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < kKeys; ++j)
+                for (int j = 0; j < NC; ++j)
                     reg_fence(v[j]);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bars->s_empty[slot]);     // the S slot may be overwritten
-                const bool full = (mask[0] & mask[1] & mask[2] & mask[3]) == 0xFFFFFFFFu;
+                uint32_t mk[NC / 32];
+#pragma unroll
+                for (int w = 0; w < NC / 32; ++w)
+                    mk[w] = kSplit ? (half ? mask[2 + w] : mask[w]) : mask[w];
+                bool full = true;
+#pragma unroll
+                for (int w = 0; w < NC / 32; ++w)
+                    full = full && mk[w] == 0xFFFFFFFFu;
+                float e = full ? tile_extreme<false, NC>(v, mk, up) : tile_extreme<true, NC>(v, mk, up);
+                if (kSplit) {
+                    const float o = exchange(e);
+                    if (!ok)
+                        break;
+                    e = up ? fmaxf(e, o) : fminf(e, o);
+                }
                 float alpha;
-                const float m_new = full ? tile_max<false>(v, mask, p.sl2, m, alpha)
-                                         : tile_max<true>(v, mask, p.sl2, m, alpha);
+                const float m_new = next_max(e, p.sl2, m, alpha);
                 // the previous tile's P.V is done: P may be overwritten and O is stable
                 if (t > 0) {
                     ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
@@ -523,27 +607,31 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
                         break;
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                        // O (TMEM, this thread's row) *= alpha, 32 columns at a time
-                        for (int c = 0; c < p.Dv / 32; ++c) {
+                        // O (TMEM, this thread's row, the warp's columns) *= alpha
+                        for (int c = o_col0; c < o_col0 + o_cols; c += 32) {
                             uint32_t o[32];
-                            tmem_ld_32x32b_x32(lane_base + kOCol + 32 * c, o);
+                            tmem_ld_32x32b_x32(lane_base + kOCol + c, o);
                             tmem_ld_wait();
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
                                 o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                            tmem_st_32x32b_x32(lane_base + kOCol + 32 * c, o);
+                            tmem_st_32x32b_x32(lane_base + kOCol + c, o);
                         }
                         tmem_st_wait();
                     }
                 }
                 float sum = 0.0f;
                 if (m_new != -INFINITY)
-                    sum = full ? tile_probs<false>(v, mask, p.sl2, m_new, pbuf, hrow)
-                               : tile_probs<true>(v, mask, p.sl2, m_new, pbuf, hrow);
+                    sum = full ? tile_probs<false, NC, kSplit>(v, mk, p.sl2, m_new, pbuf, hrow, half)
+                               : tile_probs<true, NC, kSplit>(v, mk, p.sl2, m_new, pbuf, hrow, half);
                 else
-                    for (int u = 0; u < 16; ++u)         // no key yet: P = 0
-                        *reinterpret_cast<uint4 *>(pbuf + (u >> 3) * kRows * 128 + hrow * 128 +
-                                                   ((u & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                    for (int u = 0; u < NC / 8; ++u) {    // no key yet: P = 0
+                        uint8_t *dst = pbuf + (half + (u >> 3)) * kRows * 128 + hrow * 128 +
+                                       ((u & 7) << 4);
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+                        if (kSplit)
+                            *reinterpret_cast<uint4 *>(dst + 64 * 128) = make_uint4(0u, 0u, 0u, 0u);
+                    }
                 l = l * alpha + sum;
                 m = m_new;
                 fence_proxy_async_smem();
@@ -565,6 +653,12 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
         }
         if (!ok)
             break;
+        // the row's sum over all its keys (split: both halves)
+        if (kSplit && active) {
+            l += exchange(l);
+            if (!ok)
+                break;
+        }
         // the row's last P.V, then O / l to global memory
         ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
         ok = __all_sync(0xffffffffu, ok);
@@ -573,14 +667,14 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
         tc_fence_after();
         if (active) {
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            for (int c = 0; c < p.Dv / 32; ++c) {
+            for (int c = o_col0; c < o_col0 + o_cols; c += 32) {
                 uint32_t o[32];
-                tmem_ld_32x32b_x32(lane_base + kOCol + 32 * c, o);
+                tmem_ld_32x32b_x32(lane_base + kOCol + c, o);
                 tmem_ld_wait();
                 if (hrow < p.HA) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4 *>(orow + 32 * c + j) =
+                        *reinterpret_cast<float4 *>(orow + c + j) =
                             make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
                                         __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
                 }
@@ -620,6 +714,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->row_full[s], 1);
             mbar_init(&bars->row_empty[s], 5 + kGatherWarps);   // MMA, softmax and gather warps
         }
+        for (int q = 0; q < 2; ++q)
+            for (int k = 0; k < 2; ++k)
+                mbar_init(&bars->xbar[q][k], 2);    // the pair's two warps
         mbar_init(&bars->p_full, 4);
         mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->o_empty, 4);
@@ -639,12 +736,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     WaitCtl ctl{&bars->abort, p.wait_limit};
     if (warp < 4) {
         regs_inc<kSoftmaxRegs>();
-        attn_softmax(p, smem, bars, tmem, ctl);
-    } else if (warp < 4 + kGatherWarps) {
+        if (p.split)
+            attn_softmax<true>(p, smem, bars, tmem, ctl);
+        else
+            attn_softmax<false>(p, smem, bars, tmem, ctl);
+    } else if (warp < 4 + kGatherWarps) {      // whole warpgroups
         regs_dec<kGatherRegs>();
         attn_gather(p, smem, bars, ctl);
     } else {
-        regs_dec<kCtlRegs>();
         if (warp == kMmaWarp) {
             if (lane == 0)
                 attn_mma(p, smem, bars, tmem, ctl);

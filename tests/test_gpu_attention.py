@@ -113,3 +113,11 @@ def test_attention_large_logits_rescale(lib):
     """A large scale makes later tiles exceed the running maximum by more
     than 2^8, which rescales O in tensor memory."""
     attn_case(lib, B=1, S=64, T=2048, HA=32, Dk=128, Dv=128, topk=1024, m=1, seed=11, scale=2.0)
+
+
+def test_attention_negative_scale_and_odd_heads(lib):
+    """A negative scale (the softmax then favours the smallest dot products)
+    and head counts that fill a TMEM lane quarter only in part, on both sides
+    of 64 heads (two warps share a row's keys up to 64 heads)."""
+    for HA, seed in ((48, 21), (96, 22)):
+        attn_case(lib, B=1, S=150, T=700, HA=HA, Dk=128, Dv=128, topk=300, seed=seed, scale=-0.09)
