@@ -68,6 +68,32 @@ __device__ __forceinline__ void sel_prefetch_l2(const void *src, uint32_t bytes)
                  : "memory");
 }
 
+// Calls f(key) for every key of a row's lists in global memory, with
+// kSelBatch loads per thread in flight before any of them is used: these
+// passes are bound by L2 latency, one round trip per batch instead of per key.
+constexpr int kSelBatch = 8;
+template <typename F>
+__device__ __forceinline__ void sel_for_each_key(const SelParams &sp, const uint64_t *row_lists,
+                                                 const SelSmem *sm, int tid, F &&f)
+{
+    for (int s = 0; s < sp.nsplit; ++s) {
+        const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
+        const int n = sm->split_off[s + 1] - sm->split_off[s];
+        for (int j0 = 0; j0 < n; j0 += kSelBatch * kSelThreads) {
+            uint64_t x[kSelBatch];
+#pragma unroll
+            for (int u = 0; u < kSelBatch; ++u) {
+                const int j = j0 + u * kSelThreads + tid;
+                x[u] = j < n ? __ldg(src + j) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < kSelBatch; ++u)
+                if (j0 + u * kSelThreads + tid < n)
+                    f(x[u]);
+        }
+    }
+}
+
 // For rows whose lists hold more keys than fit in registers: one histogram
 // pass over the lists in global memory (buckets = top 11 bits of the score
 // image) finds the bucket of the k-th largest key; returns the key L such that
@@ -83,17 +109,13 @@ __device__ uint64_t sel_prefilter_global(const SelParams &sp, const uint64_t *ro
     for (int i = tid; i < kSelNb; i += kSelThreads)
         sm->hist[i] = 0;
     __syncthreads();
-    for (int s = 0; s < sp.nsplit; ++s) {
-        const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
-        const int n = sm->split_off[s + 1] - sm->split_off[s];
-        for (int j = tid; j < n; j += kSelThreads) {
-            const uint32_t o = key_ord(src[j]);
-            if (b1 < 0)
-                atomicAdd(&sm->hist[o >> 21], 1u);
-            else if ((o >> 21) == static_cast<uint32_t>(b1))
-                atomicAdd(&sm->hist[(o >> 10) & (kSelNb - 1)], 1u);
-        }
-    }
+    sel_for_each_key(sp, row_lists, sm, tid, [&](uint64_t x) {
+        const uint32_t o = key_ord(x);
+        if (b1 < 0)
+            atomicAdd(&sm->hist[o >> 21], 1u);
+        else if ((o >> 21) == static_cast<uint32_t>(b1))
+            atomicAdd(&sm->hist[(o >> 10) & (kSelNb - 1)], 1u);
+    });
     __syncthreads();
     // bucket of the k-th largest, top bucket first
     constexpr int PER = kSelNb / kSelThreads;
@@ -155,15 +177,10 @@ __device__ uint64_t sel_radix_global(const SelParams &sp, const uint64_t *row_li
         for (int i = tid; i < 256; i += kSelThreads)
             sm->hist[i] = 0;
         __syncthreads();
-        for (int s = 0; s < sp.nsplit; ++s) {
-            const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
-            const int n = sm->split_off[s + 1] - sm->split_off[s];
-            for (int j = tid; j < n; j += kSelThreads) {
-                const uint64_t x = src[j];
-                if ((x & mask) == prefix)
-                    atomicAdd(&sm->hist[static_cast<uint32_t>(x >> pos) & 255u], 1u);
-            }
-        }
+        sel_for_each_key(sp, row_lists, sm, tid, [&](uint64_t x) {
+            if ((x & mask) == prefix)
+                atomicAdd(&sm->hist[static_cast<uint32_t>(x >> pos) & 255u], 1u);
+        });
         __syncthreads();
         if (tid < 32) {
             uint32_t c[8];
@@ -450,18 +467,13 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
             if (tid == 0)
                 sm->misc[2] = 0;
             __syncthreads();
-            for (int s = 0; s < sp.nsplit; ++s) {
-                const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
-                const int ns = sm->split_off[s + 1] - sm->split_off[s];
-                for (int j = tid; j < ns; j += kSelThreads) {
-                    const uint64_t x = src[j];
-                    if (x >= L) {
-                        const int slot = atomicAdd(&sm->misc[2], 1);
-                        if (CSA_CHECK_INDEX(kChkSelOut, slot, kSelKeys))
-                            sm->out[slot] = x;
-                    }
+            sel_for_each_key(sp, row_lists, sm, tid, [&](uint64_t x) {
+                if (x >= L) {
+                    const int slot = atomicAdd(&sm->misc[2], 1);
+                    if (CSA_CHECK_INDEX(kChkSelOut, slot, kSelKeys))
+                        sm->out[slot] = x;
                 }
-            }
+            });
             __syncthreads();
             if (n == n_all)
                 n = sp.topk; // the radix cut keeps exactly k
