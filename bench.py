@@ -265,11 +265,14 @@ def config_dict(wl):
 
 
 # ----------------------------------------------------------------------------- consumer leg
-def attention_leg(L, wl, out_idx, dev, stream, steps, warmup, HA=64, Dk=128, Dv=128):
+def attention_leg(L, wl, out_idx, dev, stream, steps, warmup, peaks=None, HA=64, Dk=128, Dv=128):
     """Sparse attention over the selection the timed indexer steps produced:
     CUDA-event time per call, algorithmic flops (2 HA (Dk + Dv) per selected
     key) and gathered bytes (each selected key's cache row read once per query,
-    plus q and the output)."""
+    plus q and the output).  At HA (Dk + Dv) / (Dk + Dv) / 2 ~ HA / 2 flop
+    per gathered byte the kernel sits far below the tensor/HBM ridge, so its
+    roofline is the gather: gathered bytes / time over the measured HBM copy
+    bandwidth (most gathered rows come from L2, so this can exceed 1)."""
     import torch
 
     g = torch.Generator(device=dev).manual_seed(7)
@@ -293,10 +296,15 @@ def attention_leg(L, wl, out_idx, dev, stream, steps, warmup, HA=64, Dk=128, Dv=
     ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
     flops = 2.0 * HA * (Dk + Dv) * n_sel
     gathered = n_sel * (Dk + Dv) * 2 + qa.numel() * 2 + out.numel() * 4
-    return {"kernel": "sparse_attn_kernel", "heads": HA, "Dk": Dk, "Dv": Dv,
-            "selected_keys": n_sel, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
-            "gathered_gbs": gathered / (ms * 1e-3) / 1e9,
-            "queries_per_s": wl.B * wl.S / (ms * 1e-3)}
+    gbs = gathered / (ms * 1e-3) / 1e9
+    out = {"kernel": "sparse_attn_kernel", "heads": HA, "Dk": Dk, "Dv": Dv,
+           "selected_keys": n_sel, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+           "gathered_gbs": gbs, "queries_per_s": wl.B * wl.S / (ms * 1e-3)}
+    if peaks and peaks.get("hbm_gbs"):
+        out["roofline"] = {"bound": "gather (hbm)", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                           "bytes_per_launch": gathered, "flops_per_launch": flops}
+    return out
 
 
 # ----------------------------------------------------------------------------- GPU leg
@@ -544,7 +552,7 @@ def main():
                           "ms_per_step": serial_ms,
                           "what": "upload, call and read-back of each step in series on one stream"}}
 
-    consumer = attention_leg(L, wl, out_idx, dev, stream, args.steps, args.warmup) \
+    consumer = attention_leg(L, wl, out_idx, dev, stream, args.steps, args.warmup, load_peaks()[0]) \
         if args.attention else None
 
     if rank != 0:
