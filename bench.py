@@ -622,6 +622,11 @@ def main():
         "gpu_launches": args.steps * plan.launches,
         **({"consumer": consumer} if consumer else {}),
         "plan": plan.as_dict(),
+        # extra device memory of the call: the caller's workspace (candidate lists
+        # and per-CTA score buffers, O(S*k)); the library allocates nothing else
+        "extra_memory": {"bytes": int(ws_bytes),
+                         "materialised_scores_bytes": int(wl.B * wl.S * wl.H * wl.T * 4),
+                         "per_query_bytes": ws_bytes / float(wl.B * wl.S)},
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
                     "max": max(step_ms)},
     }
