@@ -99,7 +99,7 @@ struct AttnBarriers {
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
     uint64_t s_full[2], s_empty[2];
-    uint64_t p_full, pv_done, o_empty;
+    uint64_t p_full[2], pv_done, o_empty;       // p_full: tile g's P in TMEM, entry g & 1
     uint64_t row_full[2], row_empty[2];
     uint64_t drain;
     int row_tiles[2];       // tile count of the row published in each ring entry
@@ -308,11 +308,11 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
     const uint32_t q_base = smem_u32(smem + p.off_q);
     const uint32_t k_base = smem_u32(smem + p.off_k);
     const uint32_t v_base = smem_u32(smem + p.off_v);
-    const uint32_t p_base = smem_u32(smem + p.off_p);
-    // O (+)= P(g) . V(g) for the CTA's g-th tile
+    // O (+)= P(g) . V(g) for the CTA's g-th tile; P(g) is read from TMEM, where
+    // the softmax wrote it over its own S slot (packed bf16 pairs, 64 columns)
     auto issue_pv = [&](int g, bool first) -> bool {
         const int vs = g % p.v_stages;
-        if (!wait_bounded(&bars->p_full, g & 1, ctl, kRoleMma, g) ||
+        if (!wait_bounded(&bars->p_full[g & 1], (g >> 1) & 1, ctl, kRoleMma, g) ||
             !wait_bounded(&bars->v_full[vs], (g / p.v_stages) & 1, ctl, kRoleMma, g))
             return false;
         // the row's first P.V overwrites O: the previous row's O must have been read out
@@ -322,13 +322,14 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
         fence_proxy_async_smem();                    // cp.async (generic) writes -> tensor core reads
         tc_fence_after();
         const uint32_t vst = v_base + vs * p.v_stage_bytes;
+        const uint32_t p_tmem = tmem + (g & 1) * kKeys;
 #pragma unroll
         for (int ks = 0; ks < kKeys / 16; ++ks) {
-            const uint64_t adesc = smem_desc_kmajor(p_base + (ks >> 2) * kRows * 128 + (ks & 3) * 32, 128);
             const uint64_t bdesc = smem_desc_mn_sw128(vst + ks * 16 * 128, kKeys * 128, 1024);
-            mma_f16_ss(tmem + kOCol, adesc, bdesc, idesc_pv, (!first || ks > 0) ? 1u : 0u);
+            mma_f16_ts(tmem + kOCol, p_tmem + 8 * ks, bdesc, idesc_pv, (!first || ks > 0) ? 1u : 0u);
         }
         mma_commit(&bars->v_empty[vs]);
+        mma_commit(&bars->s_empty[g & 1]);           // the slot (S, then P) is free
         mma_commit(&bars->pv_done);
         return true;
     };
@@ -349,7 +350,7 @@ __device__ void attn_mma(const AttnParams &p, uint8_t *smem, AttnBarriers *bars,
             const int slot = gt & 1;
             // P(t-1) already written while K(t) is still arriving: its P.V goes first
             bool pv_pending = t > 0;
-            if (pv_pending && mbar_try_wait(&bars->p_full, (gt - 1) & 1, false) &&
+            if (pv_pending && mbar_try_wait(&bars->p_full[(gt - 1) & 1], ((gt - 1) >> 1) & 1, false) &&
                 mbar_try_wait(&bars->v_full[(gt - 1) % p.v_stages], ((gt - 1) / p.v_stages) & 1, false) &&
                 !mbar_try_wait(&bars->k_full[ks], (gt / p.k_stages) & 1, false)) {
                 if (!(ok = issue_pv(gt - 1, gt - 1 == g0)))
@@ -436,38 +437,26 @@ __device__ __forceinline__ float next_max(float e, float sl2, float m, float &al
 }
 
 // P for a thread's NC keys: p_j = 2^(sl2 * v_j - m) (0 for masked slots),
-// rounded to bf16 and stored as 16-byte units of the K-major A operand
-// (64-key chunks of 128-byte rows, unit u of row r at ((u ^ (r & 7)) * 16),
-// chunks kRows * 128 bytes apart): the thread's keys start at chunk c0 of
-// row r, and with kDup the same units also go to row r + 64.  Returns the
-// sum of the thread's p (fp32).
-template <bool kMasked, int NC, bool kDup>
+// rounded to bf16 and packed in pairs (the lower half holds the even key), as
+// the P.V MMA reads its A operand from TMEM.  Returns the sum of the thread's
+// p (fp32).
+template <bool kMasked, int NC>
 __device__ __forceinline__ float tile_probs(const uint32_t (&v)[NC], const uint32_t (&mk)[NC / 32],
-                                            float sl2, float m, uint8_t *pbuf, int r, int c0)
+                                            float sl2, float m, uint32_t (&pk)[NC / 2])
 {
     float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const float nm = -m;
-    uint8_t *row = pbuf + c0 * kRows * 128 + r * 128;
 #pragma unroll
-    for (int u = 0; u < NC / 8; ++u) {
-        uint32_t w[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int j = 8 * u + 2 * h;
-            float p0 = ex2_approx(fmaf(__uint_as_float(v[j]), sl2, nm));
-            float p1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), sl2, nm));
-            if (kMasked) {
-                p0 = ((mk[j >> 5] >> (j & 31)) & 1u) ? p0 : 0.0f;
-                p1 = ((mk[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u) ? p1 : 0.0f;
-            }
-            s[h] += p0 + p1;
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            w[h] = *reinterpret_cast<const uint32_t *>(&b2);
+    for (int j = 0; j < NC; j += 2) {
+        float p0 = ex2_approx(fmaf(__uint_as_float(v[j]), sl2, nm));
+        float p1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), sl2, nm));
+        if (kMasked) {
+            p0 = ((mk[j >> 5] >> (j & 31)) & 1u) ? p0 : 0.0f;
+            p1 = ((mk[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u) ? p1 : 0.0f;
         }
-        uint8_t *dst = row + (u >> 3) * kRows * 128 + (((u & 7) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-        if (kDup)
-            *reinterpret_cast<uint4 *>(dst + 64 * 128) = make_uint4(w[0], w[1], w[2], w[3]);
+        s[(j >> 1) & 3] += p0 + p1;
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        pk[j / 2] = *reinterpret_cast<const uint32_t *>(&b2);
     }
     return (s[0] + s[1]) + (s[2] + s[3]);
 }
@@ -488,10 +477,11 @@ __device__ __forceinline__ void mask_slots(const AttnParams &p, int r, int t, in
 // lane quarter) and all 128 keys of a tile.  Split mode (HA <= 64, the query
 // block loaded twice so that TMEM lanes 64-127 repeat rows 0-63): warps w and
 // w ^ 2 own the same 32 head rows, w the keys 64 * (w >> 1) .. +63 of every
-// tile and the columns Dv/2 * (w >> 1) .. of O; the pair exchanges its
-// partial row maxima per tile and its partial sums per row through shared
-// memory (bounded waits on a pair barrier), and P is written to both copies
-// of each row.
+// tile; the pair exchanges its partial row maxima per tile and its partial sums
+// per row through shared memory (bounded waits on a pair barrier).  P goes to
+// TMEM over the S slot it came from (64 columns of packed bf16 pairs); in split
+// mode each copy of a row holds its own keys and zeros for the partner's, so
+// O's lanes 0-63 and 64-127 collect the two key halves, summed at the row's end.
 template <bool kSplit>
 __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *bars, uint32_t tmem,
                              const WaitCtl &ctl)
@@ -505,24 +495,37 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
     const bool active = 32 * q < p.HA;               // the warp's rows include heads
     const int rows = p.B * p.S;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int o_cols = kSplit ? p.Dv / 2 : p.Dv;     // O columns this warp rescales and writes
-    const int o_col0 = half * o_cols;
     const bool up = p.sl2 >= 0.0f;
-    uint8_t *pbuf = smem + p.off_p;
+    // split mode: partial O of the partner's output columns, [q][half][col][lane]
+    float *xo = reinterpret_cast<float *>(smem + p.off_p);
+    const int xo_cols = p.Dv / 2 < 64 ? p.Dv / 2 : 64;   // columns per exchange round
     int gt = 0, xc = 0;
     bool ok = true;
-    // pair exchange (split mode): write own value, arrive, wait for the partner's
-    auto exchange = [&](float mine) -> float {
-        float *buf = bars->xchg[xc & 1][warp];
-        buf[lane] = mine;
+    // P.V of the CTA's tile g is done.  The barrier completes one phase per
+    // P.V, and a parity wait is exact only when the barrier stands at that
+    // phase or the next: every tile waits for the previous tile's P.V before
+    // it hands over its own P, which keeps the softmax within that window
+    // (P.V(g-1) cannot start the phase after next without P(g)).
+    auto wait_pv = [&](int g) -> bool {
+        const bool good = wait_bounded(&bars->pv_done, g & 1, ctl, kRoleSoftmax, g);
+        return __all_sync(0xffffffffu, good);
+    };
+    // pair barrier (split mode): both warps of the pair have arrived
+    auto pair_sync = [&]() -> bool {
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&bars->xbar[q][xc & 1]);
         const bool good = wait_bounded(&bars->xbar[q][xc & 1], (xc >> 1) & 1, ctl, kRoleSoftmax, xc);
-        ok = __all_sync(0xffffffffu, good);
-        const float other = bars->xchg[xc & 1][warp ^ 2][lane];
         ++xc;
-        return other;
+        return __all_sync(0xffffffffu, good);
+    };
+    // pair exchange (split mode): write own value, sync, read the partner's
+    auto exchange = [&](float mine) -> float {
+        float *buf = bars->xchg[xc & 1][warp];
+        buf[lane] = mine;
+        const int x = xc & 1;
+        ok = pair_sync();
+        return bars->xchg[x][warp ^ 2][lane];
     };
     int32_t pf[4] = {-1, -1, -1, -1};             // the next tile's index slots, in flight
     if (active)
@@ -543,8 +546,9 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
         const int rn = r + gridDim.x;
         float *orow = p.out + (static_cast<size_t>(r) * p.HA + hrow) * p.Dv;
         if (nt == 0) {
+            const int c0 = kSplit ? half * (p.Dv / 2) : 0, nc = kSplit ? p.Dv / 2 : p.Dv;
             if (hrow < p.HA)
-                for (int e = o_col0; e < o_col0 + o_cols; e += 4)
+                for (int e = c0; e < c0 + nc; e += 4)
                     *reinterpret_cast<float4 *>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
             if (active && rn < rows)
                 mask_slots(p, rn, 0, lane, pf);
@@ -578,10 +582,6 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
 #pragma unroll
                 for (int j = 0; j < NC; ++j)
                     reg_fence(v[j]);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bars->s_empty[slot]);     // the S slot may be overwritten
                 uint32_t mk[NC / 32];
 #pragma unroll
                 for (int w = 0; w < NC / 32; ++w)
@@ -599,57 +599,56 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
                 }
                 float alpha;
                 const float m_new = next_max(e, p.sl2, m, alpha);
-                // the previous tile's P.V is done: P may be overwritten and O is stable
-                if (t > 0) {
-                    ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok)
+                // a raised maximum rescales O (this warp's lanes, every column)
+                // once the previous tile's P.V is done
+                if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                    if (!(ok = wait_pv(gt - 1)))
                         break;
                     tc_fence_after();
-                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                        // O (TMEM, this thread's row, the warp's columns) *= alpha
-                        for (int c = o_col0; c < o_col0 + o_cols; c += 32) {
-                            uint32_t o[32];
-                            tmem_ld_32x32b_x32(lane_base + kOCol + c, o);
-                            tmem_ld_wait();
+                    for (int c = 0; c < p.Dv; c += 32) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(lane_base + kOCol + c, o);
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                            tmem_st_32x32b_x32(lane_base + kOCol + c, o);
-                        }
-                        tmem_st_wait();
+                        for (int j = 0; j < 32; ++j)
+                            o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st_32x32b_x32(lane_base + kOCol + c, o);
                     }
                 }
+                uint32_t pk[NC / 2];
                 float sum = 0.0f;
-                if (m_new != -INFINITY)
-                    sum = full ? tile_probs<false, NC, kSplit>(v, mk, p.sl2, m_new, pbuf, hrow, half)
-                               : tile_probs<true, NC, kSplit>(v, mk, p.sl2, m_new, pbuf, hrow, half);
-                else
-                    for (int u = 0; u < NC / 8; ++u) {    // no key yet: P = 0
-                        uint8_t *dst = pbuf + (half + (u >> 3)) * kRows * 128 + hrow * 128 +
-                                       ((u & 7) << 4);
-                        *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-                        if (kSplit)
-                            *reinterpret_cast<uint4 *>(dst + 64 * 128) = make_uint4(0u, 0u, 0u, 0u);
-                    }
+                if (m_new != -INFINITY) {
+                    sum = full ? tile_probs<false, NC>(v, mk, p.sl2, m_new, pk)
+                               : tile_probs<true, NC>(v, mk, p.sl2, m_new, pk);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < NC / 2; ++j)    // no key yet: P = 0
+                        pk[j] = 0u;
+                }
                 l = l * alpha + sum;
                 m = m_new;
-                fence_proxy_async_smem();
-            } else {
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bars->s_empty[slot]);
-                if (t > 0) {
-                    ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok)
-                        break;
+                // P over the slot's first 64 columns (the S values are in registers)
+                const uint32_t pcol = lane_base + slot * kKeys;
+                if (kSplit) {
+                    uint32_t z[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        z[j] = 0u;
+                    tmem_st_32x32b_x32(pcol + 32 * half, *reinterpret_cast<uint32_t(*)[32]>(pk));
+                    tmem_st_32x32b_x32(pcol + 32 * (1 - half), z);
+                } else {
+                    tmem_st_32x32b_x32(pcol, *reinterpret_cast<uint32_t(*)[32]>(pk));
+                    tmem_st_32x32b_x32(pcol + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
                 }
+                tmem_st_wait();
             }
+            // (see wait_pv; on the first tile of a row this is the previous row's last)
+            if (gt > 0 && !(ok = wait_pv(gt - 1)))
+                break;
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars->p_full);
+                mbar_arrive(&bars->p_full[gt & 1]);
         }
         if (!ok)
             break;
@@ -660,14 +659,51 @@ __device__ void attn_softmax(const AttnParams &p, uint8_t *smem, AttnBarriers *b
                 break;
         }
         // the row's last P.V, then O / l to global memory
-        ok = wait_bounded(&bars->pv_done, (gt - 1) & 1, ctl, kRoleSoftmax, r);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok)
+        if (!(ok = wait_pv(gt - 1)))
             break;
         tc_fence_after();
-        if (active) {
-            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            for (int c = o_col0; c < o_col0 + o_cols; c += 32) {
+        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+        if (kSplit && active) {
+            // this warp writes columns half * Dv/2 ..: its own partial plus the
+            // partner's, exchanged through shared memory xo_cols at a time
+            float *mine = xo + static_cast<size_t>(q * 2 + half) * xo_cols * 32;
+            const float *theirs = xo + static_cast<size_t>(q * 2 + (1 - half)) * xo_cols * 32;
+            for (int c0 = 0; c0 < p.Dv / 2 && ok; c0 += xo_cols) {
+                // this round's columns: xo_cols, or what is left of the half
+                // (Dv is a multiple of 64, so a multiple of 32)
+                const int cw = p.Dv / 2 - c0 < xo_cols ? p.Dv / 2 - c0 : xo_cols;
+                const int pc = (1 - half) * (p.Dv / 2) + c0;   // the partner's columns
+                for (int cc = 0; cc < cw; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(lane_base + kOCol + pc + cc, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        mine[(cc + j) * 32 + lane] = __uint_as_float(o[j]);
+                }
+                if (!(ok = pair_sync()))
+                    break;
+                const int mc = half * (p.Dv / 2) + c0;         // this warp's columns
+                for (int cc = 0; cc < cw; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(lane_base + kOCol + mc + cc, o);
+                    tmem_ld_wait();
+                    if (hrow < p.HA) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4 *>(orow + mc + cc + j) = make_float4(
+                                (__uint_as_float(o[j]) + theirs[(cc + j) * 32 + lane]) * inv,
+                                (__uint_as_float(o[j + 1]) + theirs[(cc + j + 1) * 32 + lane]) * inv,
+                                (__uint_as_float(o[j + 2]) + theirs[(cc + j + 2) * 32 + lane]) * inv,
+                                (__uint_as_float(o[j + 3]) + theirs[(cc + j + 3) * 32 + lane]) * inv);
+                    }
+                }
+                ok = pair_sync();                          // the buffer may be rewritten
+            }
+            if (!ok)
+                break;
+        } else if (active) {
+            for (int c = 0; c < p.Dv; c += 32) {
                 uint32_t o[32];
                 tmem_ld_32x32b_x32(lane_base + kOCol + c, o);
                 tmem_ld_wait();
@@ -710,14 +746,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
-            mbar_init(&bars->s_empty[s], 4);
+            mbar_init(&bars->s_empty[s], 1);        // P.V of the slot's tile is done
             mbar_init(&bars->row_full[s], 1);
             mbar_init(&bars->row_empty[s], 5 + kGatherWarps);   // MMA, softmax and gather warps
         }
         for (int q = 0; q < 2; ++q)
             for (int k = 0; k < 2; ++k)
                 mbar_init(&bars->xbar[q][k], 2);    // the pair's two warps
-        mbar_init(&bars->p_full, 4);
+        for (int b = 0; b < 2; ++b)
+            mbar_init(&bars->p_full[b], 4);
         mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->o_empty, 4);
         mbar_init(&bars->drain, 1);

@@ -74,7 +74,8 @@ def test_attention_small(lib):
 
 
 def test_attention_dims(lib):
-    for Dk, Dv, HA in ((64, 64, 128), (128, 64, 16), (192, 128, 1), (256, 256, 32)):
+    for Dk, Dv, HA in ((64, 64, 128), (128, 64, 16), (192, 128, 1), (256, 256, 32),
+                       (128, 192, 40), (192, 192, 100)):
         attn_case(lib, B=1, S=70, T=300, HA=HA, Dk=Dk, Dv=Dv, topk=200, seed=Dk + Dv + HA)
 
 
