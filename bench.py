@@ -307,6 +307,50 @@ def attention_leg(L, wl, out_idx, dev, stream, steps, warmup, peaks=None, HA=64,
     return out
 
 
+def schedules_leg(L, dev, steps, warmup, n_layers=4, HA=64, Dk=128, Dv=128):
+    """One decode step of n_layers layers under each cross-layer schedule of
+    ``schedule.py`` ("own": every layer runs its own indexer then its sparse
+    attention; "mli": a layer's attention reads the previous layer's selection
+    while its own indexer runs for the next layer on a second stream;
+    "indexcache": the indexer on every second layer).  The indexer shape is
+    decode1_fp8's (32 sequences, one query each, 131,072 E4M3 keys); the
+    attention reads 128-dim bf16 key and value caches of the same length.
+    CUDA-event time of the whole step on the main stream."""
+    import torch
+    from lightning_indexer_top_02_b200 import schedule as sched
+
+    wl = workloads.CONFIGS["decode1_fp8"]
+    layers = []
+    for li in range(n_layers):
+        inp = workloads.make_inputs(wl, device=dev, seed=wl.seed + 17 * (li + 1))
+        g = torch.Generator(device=dev).manual_seed(100 + li)
+        layers.append(sched.Layer(
+            iq=inp["q"], iw=inp["w"], ik=inp["k"], ik_scale=inp["k_scale"],
+            aq=torch.randn((wl.B, wl.S, HA, Dk), generator=g, device=dev).to(torch.bfloat16),
+            kc=torch.randn((wl.B, wl.T, Dk), generator=g, device=dev).to(torch.bfloat16),
+            vc=torch.randn((wl.B, wl.T, Dv), generator=g, device=dev).to(torch.bfloat16),
+            scale=Dk ** -0.5))
+    main = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
+    out = {"layers": n_layers, "indexer": wl.name, "attention": {"heads": HA, "Dk": Dk, "Dv": Dv}}
+    for name in ("own", "mli", "indexcache"):
+        for _ in range(warmup):
+            sched.decode_layers(layers, m=wl.m, topk=wl.topk, schedule=name, main=main, side=side)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        for _ in range(steps):
+            sched.decode_layers(layers, m=wl.m, topk=wl.topk, schedule=name, main=main, side=side)
+        e1.record(main)
+        torch.cuda.synchronize(dev)
+        if L.csa_last_device_error(None) != L.CSA_OK:
+            raise SystemExit(f"device error in the {name} schedule")
+        out[name + "_ms_per_step"] = e0.elapsed_time(e1) / steps
+    out["mli_speedup_over_own"] = out["own_ms_per_step"] / out["mli_ms_per_step"]
+    out["indexcache_speedup_over_own"] = out["own_ms_per_step"] / out["indexcache_ms_per_step"]
+    return out
+
+
 # ----------------------------------------------------------------------------- GPU leg
 def main():
     ap = argparse.ArgumentParser()
@@ -328,6 +372,9 @@ def main():
     ap.add_argument("--attention", action="store_true",
                     help="also time the sparse-attention consumer over the step's selection "
                          "(HA=64 heads, Dk=Dv=128, bf16; reported under 'consumer')")
+    ap.add_argument("--schedules", action="store_true",
+                    help="also time a 4-layer decode step under the cross-layer schedules "
+                         "(own / mli / indexcache; reported under 'schedules')")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -554,6 +601,7 @@ def main():
 
     consumer = attention_leg(L, wl, out_idx, dev, stream, args.steps, args.warmup, load_peaks()[0]) \
         if args.attention else None
+    schedules = schedules_leg(L, dev, args.steps, args.warmup) if args.schedules and rank == 0 else None
 
     if rank != 0:
         if world > 1:
@@ -621,6 +669,7 @@ def main():
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * plan.launches,
         **({"consumer": consumer} if consumer else {}),
+        **({"schedules": schedules} if schedules else {}),
         "plan": plan.as_dict(),
         # extra device memory of the call: the caller's workspace (candidate lists
         # and per-CTA score buffers, O(S*k)); the library allocates nothing else
