@@ -16,23 +16,25 @@
 // last one that holds a key go through in tiles of 128:
 //   warp 13 (control): scans each row's index slots ahead of the others and
 //     publishes its tile count through a two-entry ring; loads the row's
-//     query block [128 head rows x Dk] by TMA;
+//     query block [128 head rows x Dk] by TMA (for HA <= 64 a 64-row block,
+//     loaded twice, into rows 0-63 and 64-127);
 //   warps 4-11 (gather, 16 tile rows each, two per SM sub-partition): per
-//     tile the selected key rows and
-//     value rows by cp.async, 16 bytes per thread, written straight into the
-//     128-byte-swizzled K-major layout, into separate key and value rings (a
-//     key stage frees as soon as its S is computed); every thread's arrival
-//     on the stage's barrier fires when its copies have landed;
+//     tile the selected key rows and value rows by cp.async, 16 bytes per
+//     thread, written straight into the 128-byte-swizzled K-major layout,
+//     into separate key and value rings (a key stage frees as soon as its S
+//     is computed); every thread's arrival on the stage's barrier fires when
+//     its copies have landed;
 //   warp 12 (MMA issuer, one thread; owns the TMEM allocation):
 //     S(t) = Q . K(t)^T into one of two 128-column TMEM slots (M = 128 head
-//     rows, N = 128 keys), then, once the softmax has written P(t-1),
-//     O += P(t-1) . V(t-1) into TMEM columns 256.. (N = Dv, V as an MN-major
-//     operand exactly as gathered);
+//     rows, N = 128 keys), then, once the softmax has written P(t-1) over
+//     that tile's slot, O += P(t-1) . V(t-1) with P read from TMEM (N = Dv, V
+//     as an MN-major operand exactly as gathered) into TMEM columns 256..;
+//     that P.V's completion frees the slot;
 //   warps 0-3 (softmax, thread = head row = TMEM lane): online softmax over
 //     the row's tiles in the exp2 domain with the running maximum raised only
 //     when a tile exceeds it by more than 2^8 (then O is rescaled in TMEM),
-//     P in bf16 written to shared memory as the next MMA's K-major A
-//     operand, and at the end O / l to global memory (fp32).  The tile's slot
+//     P in bf16 written back to TMEM over the first 64 columns of its S slot,
+//     and at the end O / l to global memory (fp32).  The tile's slot
 //     validity comes from index loads issued one tile ahead.
 // Head rows past HA are computed by the MMA and discarded; a softmax warp
 // whose 32 rows are all past HA only keeps the barrier protocol.  Warps 14-15
