@@ -371,7 +371,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attention", action="store_true",
                     help="also time the sparse-attention consumer over the step's selection "
-                         "(HA=64 heads, Dk=Dv=128, bf16; reported under 'consumer')")
+                         "(HA=64 heads by default, Dk=Dv=128, bf16; reported under 'consumer')")
+    ap.add_argument("--attention-heads", type=int, default=64,
+                    help="heads of the attention consumer (--attention); up to 64 heads split each "
+                         "tile's keys over warp pairs, more use one thread per head row")
     ap.add_argument("--schedules", action="store_true",
                     help="also time a 4-layer decode step under the cross-layer schedules "
                          "(own / mli / indexcache; reported under 'schedules')")
@@ -599,7 +602,8 @@ def main():
                           "ms_per_step": serial_ms,
                           "what": "upload, call and read-back of each step in series on one stream"}}
 
-    consumer = attention_leg(L, wl, out_idx, dev, stream, args.steps, args.warmup, load_peaks()[0]) \
+    consumer = attention_leg(L, wl, out_idx, dev, stream, args.steps, args.warmup, load_peaks()[0],
+                             HA=args.attention_heads) \
         if args.attention else None
     schedules = schedules_leg(L, dev, args.steps, args.warmup) if args.schedules and rank == 0 else None
 
