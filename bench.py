@@ -351,6 +351,70 @@ def schedules_leg(L, dev, steps, warmup, n_layers=4, HA=64, Dk=128, Dv=128):
     return out
 
 
+def sharded_leg(L, wl, inp, world, steps, warmup):
+    """Key-sharded selection (``sharded.py``) of this workload over ``world``
+    contiguous key ranges, one rank's share timed on this GPU: its range's
+    selection (k_local keys per query) and the exact merge of all ``world``
+    lists, against the unsharded call.  The lists' all-gather crosses NVLink on
+    real ranks; its size is reported, not timed.  Recall of the merged
+    selection against the unsharded one for exact (k_local = k) and relaxed
+    (k / 2, k / 4) local selections."""
+    import numpy as np
+    import torch
+    from lightning_indexer_top_02_b200 import sharded
+
+    q, w, k, ks = inp["q"], inp["w"], inp["k"], inp["k_scale"]
+    mode = 1 if wl.gated else 0
+
+    def timed(fn, batches=5):
+        # the median over batches of `steps` calls: a sporadic slow call
+        # (allocator, another job on the host) does not set the figure
+        for _ in range(warmup):
+            r = fn()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(batches):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                r = fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / steps)
+        return statistics.median(times), r
+
+    full_ms, (full, _) = timed(lambda: L.indexer_topk(q, w, k, k_scale=ks, m=wl.m, topk=wl.topk,
+                                                      causal=wl.causal, mode=mode))
+    f = full.cpu().numpy().reshape(-1, wl.topk)
+    out = {"ranks": world, "unsharded_ms": full_ms, "variants": []}
+    for k_local in (wl.topk, wl.topk // 2, wl.topk // 4):
+        li, ls, offs, local_ms = [], [], [], []
+        for r in range(world):
+            a, b = sharded.shard_range(wl.T, world, r)
+            kr = k[:, a:b].contiguous()
+            ksr = ks[:, a:b].contiguous() if ks is not None else None
+            ms, (i, sc) = timed(lambda: sharded.select_local(
+                q, w, kr, start=a, T_total=wl.T, m=wl.m, k_local=k_local, k_scale=ksr,
+                causal=wl.causal, mode=mode))
+            li.append(i)
+            ls.append(sc)
+            offs.append(a)
+            local_ms.append(ms)
+        merge_ms, (gi, _) = timed(lambda: sharded.merge_topk(li, ls, offs, wl.topk))
+        g = gi.cpu().numpy().reshape(-1, wl.topk)
+        rec = np.array([1.0 if np.sum(f[r] >= 0) == 0 and np.sum(g[r] >= 0) == 0 else
+                        len(np.intersect1d(g[r][g[r] >= 0], f[r][f[r] >= 0])) / max(1, np.sum(f[r] >= 0))
+                        for r in range(g.shape[0])])   # a row empty in both counts as 1
+        per_rank_ms = max(local_ms) + merge_ms
+        out["variants"].append({
+            "k_local": k_local, "local_select_ms_max": max(local_ms), "merge_ms": merge_ms,
+            "per_rank_ms_without_exchange": per_rank_ms,
+            "speedup_over_unsharded": full_ms / per_rank_ms,
+            "exchange_bytes_per_rank": int(li[0].numel() * 8 * (world - 1)),
+            "recall_mean": float(rec.mean()), "recall_min": float(rec.min())})
+    return out
+
+
 # ----------------------------------------------------------------------------- GPU leg
 def main():
     ap = argparse.ArgumentParser()
@@ -378,6 +442,9 @@ def main():
     ap.add_argument("--schedules", action="store_true",
                     help="also time a 4-layer decode step under the cross-layer schedules "
                          "(own / mli / indexcache; reported under 'schedules')")
+    ap.add_argument("--sharded", type=int, default=0, metavar="W",
+                    help="also time key-sharded selection over W key ranges, one rank's share on "
+                         "this GPU, with the recall of relaxed local selections ('sharded')")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -606,6 +673,8 @@ def main():
                              HA=args.attention_heads) \
         if args.attention else None
     schedules = schedules_leg(L, dev, args.steps, args.warmup) if args.schedules and rank == 0 else None
+    sharded_res = sharded_leg(L, wl, inp, args.sharded, args.steps, args.warmup) \
+        if args.sharded > 1 and rank == 0 else None
 
     if rank != 0:
         if world > 1:
@@ -674,6 +743,7 @@ def main():
         "gpu_launches": args.steps * plan.launches,
         **({"consumer": consumer} if consumer else {}),
         **({"schedules": schedules} if schedules else {}),
+        **({"sharded": sharded_res} if sharded_res else {}),
         "plan": plan.as_dict(),
         # extra device memory of the call: the caller's workspace (candidate lists
         # and per-CTA score buffers, O(S*k)); the library allocates nothing else

@@ -494,8 +494,21 @@ __global__ void __launch_bounds__(kSelThreads, kSelCtasPerSm)
                 const uint64_t *src = row_lists + static_cast<size_t>(s) * sp.cap;
                 const int o = sm->split_off[s];
                 const int ns = sm->split_off[s + 1] - o;
-                for (int j = tid; j < ns; j += kSelThreads)
-                    sm->out[o + j] = src[j];
+                // kSelBatch loads in flight per thread, as in sel_for_each_key
+                for (int j0 = 0; j0 < ns; j0 += kSelBatch * kSelThreads) {
+                    uint64_t x[kSelBatch];
+#pragma unroll
+                    for (int u = 0; u < kSelBatch; ++u) {
+                        const int j = j0 + u * kSelThreads + tid;
+                        x[u] = j < ns ? __ldg(src + j) : 0ull;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kSelBatch; ++u) {
+                        const int j = j0 + u * kSelThreads + tid;
+                        if (j < ns)
+                            sm->out[o + j] = x[u];
+                    }
+                }
             }
             __syncthreads();
 #pragma unroll
