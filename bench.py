@@ -429,7 +429,8 @@ def main():
                     help="query rows of the CPU-baseline sample (rank 0)")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (B, S, T, H, d, m, topk, seed, causal, "
-                         "key_fp8, gated), e.g. for a reduced profiling shape; the workload name records it")
+                         "key_fp8, gated, q_pieces, num_splits), e.g. for a reduced profiling shape; "
+                         "the workload name records it")
     ap.add_argument("--clocks-csv", default="",
                     help="keep the raw nvidia-smi clock samples of the timed region here")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -454,7 +455,7 @@ def main():
         for item in args.set:
             field, _, value = item.partition("=")
             if field not in ("B", "S", "T", "H", "d", "m", "topk", "seed", "causal", "key_fp8",
-                             "gated", "q_pieces"):
+                             "gated", "q_pieces", "num_splits"):
                 raise SystemExit(f"--set: unknown field {field!r}")
             flag = field in ("causal", "key_fp8", "gated")
             kw[field] = (value.lower() in ("1", "true")) if flag else int(value)
@@ -489,7 +490,8 @@ def main():
     out_sc = torch.empty((wl.B, wl.S, wl.topk), dtype=torch.float32, device=dev)
     mode = 1 if wl.gated else 0
     a = L.make_args(q, w, k, k_scale=ks, m=wl.m, topk=wl.topk, causal=wl.causal, mode=mode,
-                    query_pieces=wl.q_pieces, out_idx=out_idx, out_score=out_sc)
+                    query_pieces=wl.q_pieces, num_splits=wl.num_splits, out_idx=out_idx,
+                    out_score=out_sc)
     plan = L.csa_indexer_plan(a)
     ws_bytes = plan.workspace_bytes
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)

@@ -47,6 +47,7 @@ class Workload:
     gated: bool = False
     values: str = "normal"  # "normal" | "integer"
     q_pieces: int = 0       # E4M3 keys: query pieces on the tensor core (0/2 exact split, 1 one rounding)
+    num_splits: int = 0     # key-range splits per query block (0 = the library's choice)
     seed: int = 0
     note: str = ""
 
