@@ -614,7 +614,8 @@ template <> struct Ld16x256<128> {
 };
 
 // This thread's head weights for a warpgroup that reads FC columns holding FQ
-// queries: weight 2i+e belongs to column 8i + 2(lane%4) + e.
+// queries: weight 2i+e belongs to column 8i + 2(lane%4) + e.  They are held
+// halved, because the tile math multiplies them by twice the ReLU (relu2x2).
 template <int FC, int FQ>
 __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int j0, int lane,
                                             float2 (&wr)[FC / 8])
@@ -630,7 +631,7 @@ __device__ __forceinline__ void fast_load_w(const Params &p, const Item &it, int
             a = src[0];
             b = src[1];
         }
-        wr[i] = make_float2(a, b);
+        wr[i] = make_float2(0.5f * a, 0.5f * b);
     }
 }
 
@@ -650,9 +651,15 @@ __device__ __forceinline__ void fast_scale_w(const float *sig, int H, int j0, in
     }
 }
 
-__device__ __forceinline__ float2 relu2(uint32_t a, uint32_t b)
+// Twice the ReLU of a logit pair, x + |x| in one packed FP32 add: exactly 0
+// for x <= 0 and exactly 2x otherwise.  With the weights held halved, the
+// packed FMA after it forms the same exact product w * ReLU(x) as
+// max(x, 0) * w (for normal weights and |x| below half the largest float),
+// and the pair costs one instruction instead of two max operations.
+__device__ __forceinline__ float2 relu2x2(uint32_t a, uint32_t b)
 {
-    return make_float2(fmaxf(__uint_as_float(a), 0.0f), fmaxf(__uint_as_float(b), 0.0f));
+    const float x = __uint_as_float(a), y = __uint_as_float(b);
+    return __fadd2_rn(make_float2(x, y), make_float2(fabsf(x), fabsf(y)));
 }
 
 // Scores of FQ queries for one key per thread.  The warp's two 16-lane loads
@@ -690,7 +697,7 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
         const int j = i / RPQ;
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub)
-            P[sub][j] = __ffma2_rn(relu2(va[4 * i + 2 * sub], va[4 * i + 2 * sub + 1]), wr[i],
+            P[sub][j] = __ffma2_rn(relu2x2(va[4 * i + 2 * sub], va[4 * i + 2 * sub + 1]), wr[i],
                                    P[sub][j]);
     }
 #pragma unroll
@@ -713,7 +720,7 @@ __device__ __forceinline__ void fast_tile_scores(uint32_t taddr, const float2 (&
         const int j = i / RPQ;
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub)
-            P[2 + sub][j] = __ffma2_rn(relu2(vb[4 * i + 2 * sub], vb[4 * i + 2 * sub + 1]), wr[i],
+            P[2 + sub][j] = __ffma2_rn(relu2x2(vb[4 * i + 2 * sub], vb[4 * i + 2 * sub + 1]), wr[i],
                                        P[2 + sub][j]);
     }
     const bool b1 = (lane >> 1) & 1;
@@ -753,7 +760,7 @@ __device__ __forceinline__ void ft_chunk(const uint32_t (&x)[32], const float2 (
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub)
             P[2 * h + sub][j] =
-                __ffma2_rn(relu2(x[4 * r + 2 * sub], x[4 * r + 2 * sub + 1]), wr[i], P[2 * h + sub][j]);
+                __ffma2_rn(relu2x2(x[4 * r + 2 * sub], x[4 * r + 2 * sub + 1]), wr[i], P[2 * h + sub][j]);
     }
 }
 
