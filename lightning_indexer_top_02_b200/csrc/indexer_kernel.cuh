@@ -1166,6 +1166,22 @@ __device__ __forceinline__ void sel_load(const float *sj, int base, int n, int t
     }
 }
 
+// sel_load for a chunk that lies wholly below n: no bounds tests
+__device__ __forceinline__ void sel_load_full(const float *sj, int base, int tid, uint32_t (&o)[kSelPer])
+{
+    float4 x[kSelPer / 4];
+#pragma unroll
+    for (int r = 0; r < kSelPer / 4; ++r)
+        x[r] = *reinterpret_cast<const float4 *>(sj + base + r * (kGroupThreads * 4) + 4 * tid);
+#pragma unroll
+    for (int r = 0; r < kSelPer / 4; ++r) {
+        o[4 * r + 0] = ord_of_score(x[r].x);
+        o[4 * r + 1] = ord_of_score(x[r].y);
+        o[4 * r + 2] = ord_of_score(x[r].z);
+        o[4 * r + 3] = ord_of_score(x[r].w);
+    }
+}
+
 __device__ __forceinline__ int sel_index(int base, int e, int tid)
 {
     return base + (e >> 2) * (kGroupThreads * 4) + 4 * tid + (e & 3);
@@ -1182,13 +1198,17 @@ __device__ int sel_emit(const float *sj, int n, int key0, uint64_t lo, uint64_t 
     named_bar_sync(kBarSelect, kGroupThreads);
     for (int base = 0; base < n; base += kSelChunk) {
         uint32_t o[kSelPer];
-        sel_load(sj, base, n, tid, o);
+        const bool full = base + kSelChunk <= n;
+        if (full)
+            sel_load_full(sj, base, tid, o);
+        else
+            sel_load(sj, base, n, tid, o);
         uint32_t keep = 0;
         int mine = 0;
 #pragma unroll
         for (int e = 0; e < kSelPer; ++e) {
             const int i = sel_index(base, e, tid);
-            const bool k = i < n && make_key(o[e], static_cast<uint32_t>(key0 + i)) >= lo;
+            const bool k = (full || i < n) && make_key(o[e], static_cast<uint32_t>(key0 + i)) >= lo;
             keep |= k ? (1u << e) : 0u;
             mine += k;
         }
@@ -1363,11 +1383,27 @@ __device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint
     named_bar_sync(kBarSelect, kGroupThreads);
     for (int base = 0; base < n; base += kSelChunk) {
         uint32_t o[kSelPer];
-        sel_load(sj, base, n, tid, o);
+        if (base + kSelChunk <= n) {
+            // whole chunks skip the per-score bounds test, and in top-k mode
+            // (lo_ord == 0) every score passes the floor test
+            sel_load_full(sj, base, tid, o);
+            if (lo_ord == 0) {
 #pragma unroll
-        for (int e = 0; e < kSelPer; ++e)
-            if (sel_index(base, e, tid) < n && o[e] >= lo_ord)
-                atomicAdd(&sc->hist[o[e] >> kSelShift], 1u);
+                for (int e = 0; e < kSelPer; ++e)
+                    atomicAdd(&sc->hist[o[e] >> kSelShift], 1u);
+            } else {
+#pragma unroll
+                for (int e = 0; e < kSelPer; ++e)
+                    if (o[e] >= lo_ord)
+                        atomicAdd(&sc->hist[o[e] >> kSelShift], 1u);
+            }
+        } else {
+            sel_load(sj, base, n, tid, o);
+#pragma unroll
+            for (int e = 0; e < kSelPer; ++e)
+                if (sel_index(base, e, tid) < n && o[e] >= lo_ord)
+                    atomicAdd(&sc->hist[o[e] >> kSelShift], 1u);
+        }
     }
     named_bar_sync(kBarSelect, kGroupThreads);
     int bd[4];
@@ -1387,10 +1423,14 @@ __device__ int sel_query(const Params &p, const float *sj, int n, int key0, uint
         named_bar_sync(kBarSelect, kGroupThreads);
         for (int base = 0; base < n; base += kSelChunk) {
             uint32_t o[kSelPer];
-            sel_load(sj, base, n, tid, o);
+            const bool full = base + kSelChunk <= n;
+            if (full)
+                sel_load_full(sj, base, tid, o);
+            else
+                sel_load(sj, base, n, tid, o);
 #pragma unroll
             for (int e = 0; e < kSelPer; ++e)
-                if (sel_index(base, e, tid) < n && o[e] >= lo_ord && (o[e] >> kSelShift) == b1)
+                if ((full || sel_index(base, e, tid) < n) && o[e] >= lo_ord && (o[e] >> kSelShift) == b1)
                     atomicAdd(&sc->hist[(o[e] >> kSelShift2) & (kNbSelect - 1)], 1u);
         }
         named_bar_sync(kBarSelect, kGroupThreads);

@@ -21,10 +21,12 @@
 namespace csa {
 
 // Score -> unsigned integer with the same order; -0.0 is folded onto +0.0.
+// Negative scores are complemented, the rest get the sign bit set: the XOR
+// mask is the sign spread by an arithmetic shift, with bit 31 forced on.
 __device__ __forceinline__ uint32_t ord_of_score(float f)
 {
     const uint32_t b = __float_as_uint(f + 0.0f);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ float score_of_ord(uint32_t u)
