@@ -1,4 +1,4 @@
-"""Host check of the float32 identity the indexer's epilogue relies on.
+"""Host checks of the float32 identities the indexer's kernels rely on.
 
 The score of a (query, key) pair is sum_h w_h * ReLU(q_h . k) (DeepSeek-V3.2
 lightning indexer, "DeepSeek Sparse Attention" section; the CSA indexer of the
@@ -7,7 +7,9 @@ x + |x| (twice the ReLU, in one packed add) and multiplies by the weight held
 halved.  In IEEE float32 with round-to-nearest that product equals
 max(x, 0) * w bit for bit whenever w / 2 is exact (w normal) and 2x does not
 overflow; this test checks it over every class of x (both zeros, subnormals,
-normals up to half the largest float) and weights of both signs.
+normals up to half the largest float) and weights of both signs.  The
+selectors' order image (score -> unsigned integer of the same order) is
+checked the same way.
 """
 import numpy as np
 import pytest
@@ -50,3 +52,25 @@ def test_negative_logits_give_positive_zero():
     x = np.array([-0.0, -1e-45, -3.0, -np.finfo(np.float32).max], dtype=np.float32)
     twice = x + np.abs(x)
     assert np.all(twice.view(np.uint32) == 0)
+
+
+def test_order_image_is_monotone_and_folds_zero():
+    """The selectors map a float32 score to an unsigned integer of the same
+    order (negative: complement; otherwise: sign bit set) with one XOR against
+    the sign-spread mask; -0.0 is added to +0.0 first, so both zeros share one
+    image.  Checked on every class of float: the images sort like the scores."""
+    rng = np.random.default_rng(7)
+    f32 = np.finfo(np.float32)
+    bits = rng.integers(0, 1 << 32, 1 << 20, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = np.concatenate([x[np.isfinite(x)],
+                        np.array([0.0, -0.0, f32.max, -f32.max, f32.tiny, -f32.tiny,
+                                  np.inf, -np.inf], dtype=np.float32)])
+    b = (x + np.float32(0.0)).view(np.uint32)
+    spread = (b.view(np.int32) >> 31).view(np.uint32)
+    img = b ^ (spread | np.uint32(0x80000000))
+    ref = np.where(b & np.uint32(0x80000000), ~b, b | np.uint32(0x80000000))
+    assert np.array_equal(img, ref)
+    order = np.argsort(x, kind="stable")
+    assert np.all(np.diff(img[order].astype(np.int64)) >= 0)
+    assert img[x == 0.0].min() == img[x == 0.0].max()
